@@ -1,0 +1,267 @@
+// C ABI of libtlsp (declared in include/tlsp.h): argument validation,
+// workspace layout and dispatch to the kernels.
+#include <cstdio>
+
+#include "kernels.h"
+
+namespace tlsp {
+
+std::atomic<int64_t> g_launch_count{0};
+static thread_local int t_last_cuda_error = 0;
+void set_last_cuda_error(cudaError_t e) { t_last_cuda_error = (int)e; }
+
+// ----------------------------------------------------------------- workspace
+
+constexpr size_t kAlign = 256;
+constexpr size_t kStatusBytes = 256;  // status word at 0, debug flag at 64
+constexpr int64_t kPddpPartialSlots = 2048;
+
+static size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Layout {
+  size_t lse, scores, perm, tmp, seg_key, node_mu, node_v, partials, total;
+};
+
+static Layout layout_of(const tlsp_dims& d, int gs) {
+  const size_t BH = (size_t)d.batch * d.heads;
+  const size_t G = (size_t)((d.n_q + gs - 1) / gs);
+  Layout L{};
+  size_t off = kStatusBytes;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes);
+    return at;
+  };
+  L.lse = take(sizeof(float) * BH * d.n_q);
+  L.scores = take(sizeof(float) * BH * G * d.n_kv);
+  L.perm = take(sizeof(int32_t) * BH * d.n_q);
+  L.tmp = take(sizeof(int32_t) * BH * d.n_q);
+  L.seg_key = take(sizeof(uint32_t) * BH * d.n_q);
+  L.node_mu = take(sizeof(float) * BH * G * d.head_dim);
+  L.node_v = take(sizeof(float) * BH * G * d.head_dim);
+  L.partials = take(sizeof(float) * (size_t)kPddpPartialSlots *
+                    ((size_t)d.head_dim * d.head_dim + 2 * d.head_dim));
+  L.total = off;
+  return L;
+}
+
+template <class P>
+static P* at(void* ws, size_t off) {
+  return reinterpret_cast<P*>(static_cast<char*>(ws) + off);
+}
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static int validate_dims(const tlsp_dims* d) {
+  if (!d) return TLSP_ERR_INVALID_ARG;
+  if (d->batch < 1 || d->heads < 1 || d->n_q < 1 || d->n_kv < 1) return TLSP_ERR_INVALID_ARG;
+  if (d->head_dim != 64 && d->head_dim != 128) return TLSP_ERR_INVALID_ARG;
+  if (d->dtype != TLSP_F32 && d->dtype != TLSP_BF16) return TLSP_ERR_INVALID_ARG;
+  if ((int64_t)d->batch * d->heads > 65535) return TLSP_ERR_UNSUPPORTED;
+  return TLSP_OK;
+}
+
+static int validate_grouping(const tlsp_dims* d, int32_t gs) {
+  if (gs < 1) return TLSP_ERR_INVALID_ARG;
+  const int64_t G = (d->n_q + (int64_t)gs - 1) / gs;
+  if (G > 65535) return TLSP_ERR_UNSUPPORTED;
+  return TLSP_OK;
+}
+
+static int check_ws(const tlsp_dims* d, int32_t gs, void* ws, size_t ws_bytes) {
+  if (!ws || !aligned16(ws)) return TLSP_ERR_INVALID_ARG;
+  if (ws_bytes < layout_of(*d, gs).total) return TLSP_ERR_WORKSPACE;
+  return TLSP_OK;
+}
+
+static AttnArgs attn_args(const tlsp_dims* d, const void* Q, const void* K, const void* V,
+                          int32_t gs, int32_t k, void* ws) {
+  AttnArgs a;
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.BH = (int64_t)d->batch * d->heads;
+  a.n_q = d->n_q;
+  a.n_kv = d->n_kv;
+  a.d = d->head_dim;
+  a.gs = gs;
+  a.G = (d->n_q + gs - 1) / gs;
+  a.k = k;
+  a.bf16 = d->dtype == TLSP_BF16;
+  a.status = at<int>(ws, 0);
+  return a;
+}
+
+__global__ void bounded_wait_kernel(volatile int* flag, int* status, int64_t spin_limit) {
+  for (int64_t i = 0; i < spin_limit; ++i) {
+    if (*flag != 0) return;
+    __nanosleep(32);
+  }
+  record_status(status, TLSP_ERR_TIMEOUT);
+}
+
+static int group_impl(const tlsp_dims* dims, const void* Q, int32_t gs, int32_t* groups,
+                      float* proj, void* ws, size_t ws_bytes, void* stream) {
+  TLSP_TRY(validate_dims(dims));
+  TLSP_TRY(validate_grouping(dims, gs));
+  if (!Q || !groups || !aligned16(Q)) return TLSP_ERR_INVALID_ARG;
+  TLSP_TRY(check_ws(dims, gs, ws, ws_bytes));
+  const Layout L = layout_of(*dims, gs);
+  const int64_t BH = (int64_t)dims->batch * dims->heads;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (proj) {
+    const int levels = tlsp_num_levels(dims->n_q, gs);
+    if (levels > 0) {
+      cudaError_t e = cudaMemsetAsync(proj, 0, sizeof(float) * levels * BH * dims->n_q, st);
+      if (e != cudaSuccess) {
+        set_last_cuda_error(e);
+        return TLSP_ERR_CUDA;
+      }
+    }
+  }
+  PddpWork w{at<int32_t>(ws, L.perm),    at<int32_t>(ws, L.tmp),   at<uint32_t>(ws, L.seg_key),
+             at<float>(ws, L.node_mu),   at<float>(ws, L.node_v),  at<float>(ws, L.partials),
+             kPddpPartialSlots};
+  return run_pddp(Q, dims->dtype == TLSP_BF16, dims->head_dim, BH, dims->n_q, gs, groups, proj, w,
+                  st);
+}
+
+}  // namespace tlsp
+
+using namespace tlsp;
+
+extern "C" {
+
+int32_t tlsp_num_groups(int32_t n_q, int32_t group_size) {
+  if (n_q < 1 || group_size < 1) return -1;
+  return (int32_t)(((int64_t)n_q + group_size - 1) / group_size);
+}
+
+int32_t tlsp_num_levels(int32_t n_q, int32_t group_size) {
+  const int32_t G = tlsp_num_groups(n_q, group_size);
+  if (G < 1) return -1;
+  int32_t L = 0;
+  while ((int64_t(1) << L) < G) ++L;
+  return L;
+}
+
+size_t tlsp_workspace_bytes(const tlsp_dims* dims, int32_t group_size, int32_t k) {
+  if (validate_dims(dims) != TLSP_OK || validate_grouping(dims, group_size) != TLSP_OK) return 0;
+  if (k < 1 || k > dims->n_kv) return 0;
+  return layout_of(*dims, group_size).total;
+}
+
+int tlsp_group_queries(const tlsp_dims* dims, const void* Q, int32_t group_size, int32_t* groups,
+                       void* ws, size_t ws_bytes, void* stream) {
+  return group_impl(dims, Q, group_size, groups, nullptr, ws, ws_bytes, stream);
+}
+
+int tlsp_group_queries_trace(const tlsp_dims* dims, const void* Q, int32_t group_size,
+                             int32_t* groups, float* proj, void* ws, size_t ws_bytes,
+                             void* stream) {
+  if (!proj) return TLSP_ERR_INVALID_ARG;
+  return group_impl(dims, Q, group_size, groups, proj, ws, ws_bytes, stream);
+}
+
+int tlsp_split_from_projections(const float* proj, const int32_t* members, int32_t n,
+                                int32_t n_left, int32_t* left_out, int32_t* right_out,
+                                void* ws, size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (!proj || !members || n < 1 || n_left < 0 || n_left > n) return TLSP_ERR_INVALID_ARG;
+  if ((n_left > 0 && !left_out) || (n_left < n && !right_out)) return TLSP_ERR_INVALID_ARG;
+  return launch_split(proj, members, n, n_left, left_out, right_out, (cudaStream_t)stream);
+}
+
+int tlsp_anchor_attention(const tlsp_dims* dims, const void* Q, const void* K, const void* V,
+                          const int32_t* groups, int32_t group_size, int32_t k, void* O,
+                          int32_t* indices, float* R, float* scores, void* ws, size_t ws_bytes,
+                          void* stream) {
+  TLSP_TRY(validate_dims(dims));
+  TLSP_TRY(validate_grouping(dims, group_size));
+  if (k < 1 || k > dims->n_kv) return TLSP_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !groups || !O || !indices || !R) return TLSP_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(R))
+    return TLSP_ERR_INVALID_ARG;
+  TLSP_TRY(check_ws(dims, group_size, ws, ws_bytes));
+  const Layout L = layout_of(*dims, group_size);
+  cudaStream_t st = (cudaStream_t)stream;
+  const AttnArgs a = attn_args(dims, Q, K, V, group_size, k, ws);
+  float* lse = at<float>(ws, L.lse);
+  float* S = scores ? scores : at<float>(ws, L.scores);
+  TLSP_TRY(simt_dense(a, O, lse, st));
+  TLSP_TRY(simt_scores(a, groups, lse, S, st));
+  TLSP_TRY(launch_topk(S, a.BH * a.G, a.n_kv, k, indices, st));
+  return simt_sparse(a, groups, indices, O, R, nullptr, nullptr, st);
+}
+
+int tlsp_reuse_attention(const tlsp_dims* dims, const void* Q, const void* K, const void* V,
+                         const int32_t* groups, int32_t group_size, int32_t k,
+                         const int32_t* indices, const float* R, void* O, void* ws,
+                         size_t ws_bytes, void* stream) {
+  TLSP_TRY(validate_dims(dims));
+  TLSP_TRY(validate_grouping(dims, group_size));
+  if (k < 1 || k > dims->n_kv) return TLSP_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !groups || !O || !indices || !R) return TLSP_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(R))
+    return TLSP_ERR_INVALID_ARG;
+  TLSP_TRY(check_ws(dims, group_size, ws, ws_bytes));
+  const AttnArgs a = attn_args(dims, Q, K, V, group_size, k, ws);
+  return simt_sparse(a, groups, indices, nullptr, nullptr, R, O, (cudaStream_t)stream);
+}
+
+int tlsp_topk_from_scores(const float* scores, int32_t rows, int32_t n_kv, int32_t k,
+                          int32_t* indices, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (!scores || !indices || rows < 0 || n_kv < 1 || k < 1 || k > n_kv)
+    return TLSP_ERR_INVALID_ARG;
+  return launch_topk(scores, rows, n_kv, k, indices, (cudaStream_t)stream);
+}
+
+int tlsp_get_device_status(const void* ws) {
+  if (!ws) return TLSP_ERR_INVALID_ARG;
+  int code = 0;
+  cudaError_t e = cudaMemcpy(&code, ws, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) {
+    set_last_cuda_error(e);
+    return TLSP_ERR_CUDA;
+  }
+  return code;
+}
+
+int tlsp_reset_device_status(void* ws, void* stream) {
+  if (!ws) return TLSP_ERR_INVALID_ARG;
+  cudaError_t e = cudaMemsetAsync(ws, 0, kStatusBytes, (cudaStream_t)stream);
+  if (e != cudaSuccess) {
+    set_last_cuda_error(e);
+    return TLSP_ERR_CUDA;
+  }
+  return TLSP_OK;
+}
+
+int tlsp_debug_bounded_wait(void* ws, size_t ws_bytes, int64_t spin_limit, void* stream) {
+  if (!ws || ws_bytes < kStatusBytes || spin_limit < 0) return TLSP_ERR_INVALID_ARG;
+  bounded_wait_kernel<<<1, 1, 0, (cudaStream_t)stream>>>(at<volatile int>(ws, 64), at<int>(ws, 0),
+                                                         spin_limit);
+  return check_launch();
+}
+
+const char* tlsp_status_string(int status) {
+  switch (status) {
+    case TLSP_OK: return "TLSP_OK";
+    case TLSP_ERR_INVALID_ARG: return "TLSP_ERR_INVALID_ARG";
+    case TLSP_ERR_UNSUPPORTED: return "TLSP_ERR_UNSUPPORTED";
+    case TLSP_ERR_WORKSPACE: return "TLSP_ERR_WORKSPACE";
+    case TLSP_ERR_CUDA: return "TLSP_ERR_CUDA";
+    case TLSP_ERR_TIMEOUT: return "TLSP_ERR_TIMEOUT";
+    case TLSP_ERR_DEVICE_ASSERT: return "TLSP_ERR_DEVICE_ASSERT";
+    default: return "TLSP_UNKNOWN_STATUS";
+  }
+}
+
+int tlsp_last_cuda_error(void) { return t_last_cuda_error; }
+
+int64_t tlsp_launch_count(void) { return g_launch_count.load(); }
+
+}  // extern "C"

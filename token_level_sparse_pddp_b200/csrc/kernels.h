@@ -1,0 +1,42 @@
+// Internal interface between the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include "common.cuh"
+
+namespace tlsp {
+
+// ---- pddp.cu: tile-aligned query grouping
+struct PddpWork {
+  int32_t* perm;      // [BH, n_q] token ids, node segments contiguous
+  int32_t* tmp;       // [BH, n_q] partition scratch
+  uint32_t* seg_key;  // [BH, n_q] order keys of the projections, by position
+  float* node_mu;     // [BH, G, d]
+  float* node_v;      // [BH, G, d]
+  float* partials;    // [partial_slots, d*d + 2d] chunk moments
+  int64_t partial_slots;
+};
+int run_pddp(const void* Q, bool bf16, int d, int64_t BH, int n_q, int gs, int32_t* groups,
+             float* trace, const PddpWork& w, cudaStream_t st);
+
+// ---- select.cu: top-k and the single PDDP cut
+int launch_topk(const float* scores, int64_t rows, int n_kv, int k, int32_t* indices,
+                cudaStream_t stream);
+int launch_split(const float* proj, const int32_t* members, int n, int n_left, int32_t* left,
+                 int32_t* right, cudaStream_t stream);
+
+// ---- attention kernels
+struct AttnArgs {
+  const void *Q, *K, *V;
+  int64_t BH;
+  int n_q, n_kv, d, gs, G, k;
+  bool bf16;
+  int* status;
+};
+int simt_dense(const AttnArgs& a, void* O, float* LSE, cudaStream_t st);
+int simt_scores(const AttnArgs& a, const int32_t* groups, const float* LSE, float* S,
+                cudaStream_t st);
+int simt_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices,
+                const void* O_full, float* R_out, const float* R_in, void* O_out,
+                cudaStream_t st);
+
+}  // namespace tlsp
