@@ -80,9 +80,9 @@ int32_t tlsp_num_levels(int32_t n_q, int32_t group_size);
  * NULL `scores` argument is always allowed. */
 size_t tlsp_workspace_bytes(const tlsp_dims* dims, int32_t group_size, int32_t k);
 
-/* Tile-aligned query grouping by fast PDDP (review section 3: "similar
- * queries are grouped into equal-size tile-aligned groups with fast principal
- * direction divisive partitioning").
+/* Tile-aligned query grouping by fast PDDP (review section 3: queries that
+ * look alike share a group; groups have equal size, aligned to the GPU tile,
+ * and are formed by principal direction divisive partitioning).
  *   Q       [B, H, n_q, d] in dims->dtype (the anchor step's queries).
  *   groups  out, int32 [B, H, G*group_size]: group g occupies
  *           [g*group_size, (g+1)*group_size); token ids ascending inside a
@@ -137,6 +137,15 @@ int tlsp_anchor_attention(const tlsp_dims* dims, const void* Q, const void* K, c
                           const int32_t* groups, int32_t group_size, int32_t k, void* O,
                           int32_t* indices, float* R, float* scores, void* ws, size_t ws_bytes,
                           void* stream);
+
+/* Dense attention alone (the dense pass of the anchor step; also the
+ * baseline a reuse step is compared with).
+ *   O    out [B, H, n_q, d] in dims->dtype: softmax(q_i . k_j / sqrt(d)) V.
+ *   lse  optional out fp32 [B, H, n_q]: log sum_j exp(q_i . k_j / sqrt(d))
+ *        (NULL: kept in the workspace, which must then hold at least
+ *        256 + 4*B*H*n_q bytes; with lse given, 256 bytes suffice). */
+int tlsp_dense_attention(const tlsp_dims* dims, const void* Q, const void* K, const void* V,
+                         void* O, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /* Reuse step (review section 3: reuse of the anchor's exact selections and
  * the residual as an additive correction).

@@ -195,6 +195,18 @@ int tlsp_anchor_attention(const tlsp_dims* dims, const void* Q, const void* K, c
   return simt_sparse(a, groups, indices, O, R, nullptr, nullptr, st);
 }
 
+int tlsp_dense_attention(const tlsp_dims* dims, const void* Q, const void* K, const void* V,
+                         void* O, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  TLSP_TRY(validate_dims(dims));
+  if (!Q || !K || !V || !O) return TLSP_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return TLSP_ERR_INVALID_ARG;
+  if (!ws || !aligned16(ws)) return TLSP_ERR_INVALID_ARG;
+  const size_t lse_bytes = sizeof(float) * (size_t)dims->batch * dims->heads * dims->n_q;
+  if (ws_bytes < kStatusBytes + (lse ? 0 : lse_bytes)) return TLSP_ERR_WORKSPACE;
+  const AttnArgs a = attn_args(dims, Q, K, V, 1, 1, ws);
+  return simt_dense(a, O, lse ? lse : at<float>(ws, kStatusBytes), (cudaStream_t)stream);
+}
+
 int tlsp_reuse_attention(const tlsp_dims* dims, const void* Q, const void* K, const void* V,
                          const int32_t* groups, int32_t group_size, int32_t k,
                          const int32_t* indices, const float* R, void* O, void* ws,

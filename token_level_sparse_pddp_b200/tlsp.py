@@ -30,7 +30,7 @@ TLSP_BF16 = 1
 EXPORTED = [
     "tlsp_num_groups", "tlsp_num_levels", "tlsp_workspace_bytes", "tlsp_group_queries",
     "tlsp_group_queries_trace", "tlsp_split_from_projections", "tlsp_anchor_attention",
-    "tlsp_reuse_attention", "tlsp_topk_from_scores", "tlsp_get_device_status",
+    "tlsp_reuse_attention", "tlsp_dense_attention", "tlsp_topk_from_scores", "tlsp_get_device_status",
     "tlsp_reset_device_status", "tlsp_debug_bounded_wait", "tlsp_status_string",
     "tlsp_last_cuda_error", "tlsp_launch_count",
 ]
@@ -71,6 +71,7 @@ def lib() -> ctypes.CDLL:
                                       [dp, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, sz, vp]),
             "tlsp_reuse_attention": (ctypes.c_int,
                                      [dp, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]),
+            "tlsp_dense_attention": (ctypes.c_int, [dp, vp, vp, vp, vp, vp, vp, sz, vp]),
             "tlsp_topk_from_scores": (ctypes.c_int, [vp, i32, i32, i32, vp, vp, sz, vp]),
             "tlsp_get_device_status": (ctypes.c_int, [vp]),
             "tlsp_reset_device_status": (ctypes.c_int, [vp, vp]),
@@ -158,11 +159,13 @@ class Workspace:
         _check(lib().tlsp_reset_device_status(self.ptr, _stream()), "tlsp_reset_device_status")
 
 
-def group_queries(Q: torch.Tensor, group_size: int, ws: Workspace, trace: bool = False):
+def group_queries(Q: torch.Tensor, group_size: int, ws: Workspace, trace: bool = False,
+                  out: Optional[torch.Tensor] = None):
     """PDDP grouping -> groups int32 [B, H, G*group_size] (and per-level projections)."""
     d = dims_of(Q)
     G = num_groups(d.n_q, group_size)
-    groups = torch.empty((d.batch, d.heads, G * group_size), dtype=torch.int32, device=Q.device)
+    groups = (torch.empty((d.batch, d.heads, G * group_size), dtype=torch.int32, device=Q.device)
+              if out is None else out)
     if trace:
         L = num_levels(d.n_q, group_size)
         proj = torch.empty((max(L, 0), d.batch, d.heads, d.n_q), dtype=torch.float32,
@@ -205,6 +208,16 @@ def reuse_attention(Q, K, V, groups, group_size: int, k: int, indices, R, ws: Wo
     _check(lib().tlsp_reuse_attention(ctypes.byref(d), _ptr(Q), _ptr(K), _ptr(V), _ptr(groups),
                                       group_size, k, _ptr(indices), _ptr(R), _ptr(O), ws.ptr,
                                       ws.nbytes, _stream()), "tlsp_reuse_attention")
+    return O
+
+
+def dense_attention(Q, K, V, ws: Workspace, out=None, lse=None):
+    """Dense attention alone -> O (and fills lse [B, H, n_q] if given)."""
+    d = dims_of(Q, K)
+    O = torch.empty_like(Q) if out is None else out
+    _check(lib().tlsp_dense_attention(ctypes.byref(d), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
+                                      _ptr(lse), ws.ptr, ws.nbytes, _stream()),
+           "tlsp_dense_attention")
     return O
 
 
