@@ -192,7 +192,7 @@ int tlsp_anchor_attention(const tlsp_dims* dims, const void* Q, const void* K, c
   TLSP_TRY(simt_dense(a, O, lse, st));
   TLSP_TRY(simt_scores(a, groups, lse, S, st));
   TLSP_TRY(launch_topk(S, a.BH * a.G, a.n_kv, k, indices, st));
-  return simt_sparse(a, groups, indices, O, R, nullptr, nullptr, st);
+  return sparse_pass(a, groups, indices, O, R, nullptr, nullptr, st);
 }
 
 int tlsp_dense_attention(const tlsp_dims* dims, const void* Q, const void* K, const void* V,
@@ -219,7 +219,7 @@ int tlsp_reuse_attention(const tlsp_dims* dims, const void* Q, const void* K, co
     return TLSP_ERR_INVALID_ARG;
   TLSP_TRY(check_ws(dims, group_size, ws, ws_bytes));
   const AttnArgs a = attn_args(dims, Q, K, V, group_size, k, ws);
-  return simt_sparse(a, groups, indices, nullptr, nullptr, R, O, (cudaStream_t)stream);
+  return sparse_pass(a, groups, indices, nullptr, nullptr, R, O, (cudaStream_t)stream);
 }
 
 int tlsp_topk_from_scores(const float* scores, int32_t rows, int32_t n_kv, int32_t k,

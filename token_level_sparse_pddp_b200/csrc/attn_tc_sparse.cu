@@ -1,0 +1,403 @@
+// Gathered sparse attention on the sm_100a tensor cores (bf16, head_dim 128),
+// with the dense-sparse residual fused into the epilogue.
+//
+// MC-Sparse review, section 3: each query group attends only to its own
+// selected KV tokens (token level, beyond block boundaries). On the anchor
+// step the epilogue stores R = O_full - O_sparse; on reuse steps it returns
+// O_sparse + R (additive correction for the discarded tail).
+//
+// One CTA per 128-query tile of a group (a group of g_s <= 128 queries is one
+// tile; the padding rows of a ragged group are zero and never written back).
+// Warp roles:
+//   warps 0-3  softmax + epilogue: thread t owns query row t = TMEM lane t;
+//   warps 4-7  producers: gather the tile's Q rows and, 128 selected keys at
+//              a time, the K and V rows with 16-byte cp.async into 128-byte
+//              swizzled shared memory (the tcgen05 canonical layout);
+//   warp 8     allocates TMEM; lane 0 issues the tcgen05.mma instructions.
+// Per chunk j of 128 keys: S_j = Q K_j^T (M=N=K=128, fp32 in TMEM), online
+// softmax with exp2 on the SFU, P_j (bf16) written back to TMEM, and
+// O += P_j V_j with A read from TMEM and V as an MN-major B operand.
+// TMEM columns: S double buffer [0,256), O [256,384), P double buffer
+// [384,512). K and V have two shared-memory slots each, so the gather of
+// chunk j+2 overlaps the math of chunks j and j+1.
+// The running max is only raised when it grows by more than 2^8 (then O is
+// rescaled in TMEM); between raises the stale max is used for both the
+// numerator and the denominator, which cancels exactly in O / l.
+// Every wait is bounded (1 s); on expiry the kernel records
+// TLSP_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
+#include "kernels.h"
+#include "tc_ptx.cuh"
+
+namespace tlsp {
+namespace {
+
+constexpr int kTile = 128;
+constexpr int kD = 128;
+constexpr int kThreads = 288;
+constexpr uint32_t kTileBytes = kTile * kD * 2;  // 32 KB
+constexpr uint32_t kHalfBytes = kTileBytes / 2;  // one 64-column half: 128 rows x 128 B
+constexpr uint32_t kSmQ = 0;
+constexpr uint32_t kSmK = kTileBytes;      // 2 slots
+constexpr uint32_t kSmV = 3 * kTileBytes;  // 2 slots
+constexpr uint32_t kSmBar = 5 * kTileBytes;
+constexpr uint32_t kSmemBytes = kSmBar + 256 + 1024;  // + slack to align the base to 1024 B
+constexpr uint32_t kTmCols = 512;
+constexpr uint32_t kTmS = 0, kTmO = 256, kTmP = 384;
+constexpr uint64_t kWaitNs = 1000000000ull;
+constexpr float kRescaleLog2 = 8.f;
+
+struct Bars {
+  uint64_t q_full;
+  uint64_t k_full[2], v_full[2], k_empty[2], v_empty[2];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_done, o_final, drain;
+  uint32_t tmem_base;
+  int abort;
+};
+static_assert(sizeof(Bars) <= 256, "barrier block");
+
+struct SparseParams {
+  const __nv_bfloat16* Q;
+  const __nv_bfloat16* K;
+  const __nv_bfloat16* V;
+  const int32_t* groups;
+  const int32_t* indices;
+  int n_q, n_kv, gs, G, k, tiles_per_group;
+  float scale_log2;
+  const __nv_bfloat16* O_full;
+  float* R_out;
+  const float* R_in;
+  __nv_bfloat16* O_out;
+  int* status;
+};
+
+// Row r (0..127) of a [128 x 128] bf16 tile, 16-byte chunk c (0..15), in
+// the 128-byte-swizzled layout: two 64-column halves of 128 rows x 128 B,
+// chunk index XOR (row mod 8) inside each 1024-byte atom.
+__device__ __forceinline__ uint32_t swz(int r, int c) {
+  return (uint32_t)(c >> 3) * kHalfBytes + (uint32_t)r * 128u + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
+}
+
+// 16 copies per producer thread: 128 rows x 16 chunks; consecutive threads
+// take consecutive chunks of a row (two 256-byte rows per warp instruction).
+template <class RowOf>
+__device__ __forceinline__ void gather_tile(uint32_t dst, const __nv_bfloat16* src, RowOf row_of,
+                                            int p) {
+#pragma unroll 4
+  for (int it = 0; it < 16; ++it) {
+    const int lin = it * 128 + p;
+    const int r = lin >> 4, c = lin & 15;
+    const int row = row_of(r);
+    const __nv_bfloat16* s = src + (row >= 0 ? (int64_t)row * kD + c * 8 : 0);
+    ptx::cp_async16(dst + swz(r, c), s, row >= 0 ? 16u : 0u);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ void fail(Bars& b, int* status) {
+  b.abort = 1;
+  record_status(status, TLSP_ERR_TIMEOUT);
+}
+
+template <bool kAnchor>
+__global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparseParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = ptx::smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw);
+  Bars& bars = *reinterpret_cast<Bars*>(smem + kSmBar);
+  volatile int* abort_flag = &bars.abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tiles_per_head = p.G * p.tiles_per_group;
+  const int64_t bh = blockIdx.x / tiles_per_head;
+  const int rem = blockIdx.x % tiles_per_head;
+  const int g = rem / p.tiles_per_group, t = rem % p.tiles_per_group;
+  const int32_t* grp = p.groups + (bh * p.G + g) * (int64_t)p.gs;
+  const int32_t* sel = p.indices + (bh * p.G + g) * (int64_t)p.k;
+  const int n_chunks = (p.k + kTile - 1) / kTile;
+
+  if (tid == 0) {
+    ptx::mbar_init(&bars.q_full, 128);
+    for (int s = 0; s < 2; ++s) {
+      ptx::mbar_init(&bars.k_full[s], 128);
+      ptx::mbar_init(&bars.v_full[s], 128);
+      ptx::mbar_init(&bars.k_empty[s], 1);
+      ptx::mbar_init(&bars.v_empty[s], 1);
+      ptx::mbar_init(&bars.s_full[s], 1);
+      ptx::mbar_init(&bars.p_full[s], 128);
+    }
+    ptx::mbar_init(&bars.o_done, 1);
+    ptx::mbar_init(&bars.o_final, 1);
+    ptx::mbar_init(&bars.drain, 1);
+    bars.abort = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 8) {
+    ptx::tmem_alloc(&bars.tmem_base, kTmCols);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+
+  if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ producers
+    const int pt = tid - 128;
+    const __nv_bfloat16* Qbh = p.Q + bh * (int64_t)p.n_q * kD;
+    const __nv_bfloat16* Kbh = p.K + bh * (int64_t)p.n_kv * kD;
+    const __nv_bfloat16* Vbh = p.V + bh * (int64_t)p.n_kv * kD;
+    gather_tile(base + kSmQ, Qbh, [&](int r) -> int {
+      const int gr = t * kTile + r;
+      if (gr >= p.gs) return -1;
+      const int tok = grp[gr];
+      if (tok >= p.n_q) {
+        record_status(p.status, TLSP_ERR_DEVICE_ASSERT);
+        return -1;
+      }
+      return tok;
+    }, pt);
+    ptx::cp_async_arrive_noinc(&bars.q_full);
+    for (int j = 0; j < n_chunks; ++j) {
+      const int s = j & 1;
+      auto kv_row = [&](int r) -> int {
+        const int q = j * kTile + r;
+        if (q >= p.k) return -1;
+        const int kv = __ldg(sel + q);
+        if ((unsigned)kv >= (unsigned)p.n_kv) {
+          record_status(p.status, TLSP_ERR_DEVICE_ASSERT);
+          return -1;
+        }
+        return kv;
+      };
+      if (j >= 2 && !ptx::mbar_wait(&bars.k_empty[s], ((j >> 1) - 1) & 1, abort_flag, kWaitNs)) {
+        fail(bars, p.status);
+        break;
+      }
+      gather_tile(base + kSmK + s * kTileBytes, Kbh, kv_row, pt);
+      ptx::cp_async_arrive_noinc(&bars.k_full[s]);
+      if (j >= 2 && !ptx::mbar_wait(&bars.v_empty[s], ((j >> 1) - 1) & 1, abort_flag, kWaitNs)) {
+        fail(bars, p.status);
+        break;
+      }
+      gather_tile(base + kSmV + s * kTileBytes, Vbh, kv_row, pt);
+      ptx::cp_async_arrive_noinc(&bars.v_full[s]);
+    }
+    ptx::cp_async_wait_all();
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t id_qk = ptx::idesc_bf16(kTile, kTile, false);
+      constexpr uint32_t id_pv = ptx::idesc_bf16(kTile, kD, true);
+      bool ok = ptx::mbar_wait(&bars.q_full, 0, abort_flag, kWaitNs);
+      auto issue_qk = [&](int j) {
+        const int s = j & 1;
+        ok = ok && ptx::mbar_wait(&bars.k_full[s], (j >> 1) & 1, abort_flag, kWaitNs);
+        if (!ok) return;
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_after();
+        const uint32_t kb = base + kSmK + s * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32u;
+          ptx::mma_ss(tmem + kTmS + s * kTile, ptx::sw128_desc(base + kSmQ + off, 16, 1024),
+                      ptx::sw128_desc(kb + off, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
+        }
+        ptx::tc_commit(&bars.s_full[s]);
+        ptx::tc_commit(&bars.k_empty[s]);
+      };
+      issue_qk(0);
+      if (n_chunks > 1) issue_qk(1);
+      for (int j = 0; j < n_chunks && ok; ++j) {
+        const int s = j & 1;
+        ok = ptx::mbar_wait(&bars.p_full[s], (j >> 1) & 1, abort_flag, kWaitNs) &&
+             ptx::mbar_wait(&bars.v_full[s], (j >> 1) & 1, abort_flag, kWaitNs);
+        if (!ok) break;
+        ptx::fence_proxy_async_smem();
+        ptx::tc_fence_after();
+        const uint32_t vb = base + kSmV + s * kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          ptx::mma_ts(tmem + kTmO, tmem + kTmP + s * 64 + kk * 8,
+                      ptx::sw128_desc(vb + kk * 2048, kHalfBytes, 1024), id_pv,
+                      (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        ptx::tc_commit(&bars.v_empty[s]);
+        ptx::tc_commit(j == n_chunks - 1 ? &bars.o_final : &bars.o_done);
+        if (j + 2 < n_chunks) issue_qk(j + 2);
+      }
+      if (!ok) fail(bars, p.status);
+      // all issued MMAs must land before TMEM is released
+      ptx::tc_commit(&bars.drain);
+      ptx::mbar_wait(&bars.drain, 0, abort_flag, kWaitNs);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int r = tid;
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const int gr = t * kTile + r;
+    int tok = gr < p.gs ? grp[gr] : -1;
+    if (tok >= p.n_q) tok = -1;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_chunks; ++j) {
+      const int s = j & 1;
+      if (!ptx::mbar_wait(&bars.s_full[s], (j >> 1) & 1, abort_flag, kWaitNs)) {
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      uint32_t a[4][32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) ptx::tmem_ld32(tl + kTmS + s * kTile + q * 32, a[q]);
+      ptx::tmem_ld_wait(a[0]);
+      ptx::reg_barrier(a[1]);
+      ptx::reg_barrier(a[2]);
+      ptx::reg_barrier(a[3]);
+      const int valid_n = min(kTile, p.k - j * kTile);
+      float mx = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (q * 32 + e < valid_n) mx = fmaxf(mx, __uint_as_float(a[q][e]));
+      const float m_tile = mx * p.scale_log2;
+      if (m_tile > m_run + kRescaleLog2) {
+        if (j > 0) {
+          // raise the reference max: O *= 2^(m_run - m_tile) once PV(j-1) has landed
+          const float f = ptx::ex2(m_run - m_tile);
+          if (!ptx::mbar_wait(&bars.o_done, (j - 1) & 1, abort_flag, kWaitNs)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+#pragma unroll 1
+          for (int q = 0; q < 4; ++q) {
+            uint32_t o[32];
+            ptx::tmem_ld32(tl + kTmO + q * 32, o);
+            ptx::tmem_ld_wait(o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            ptx::tmem_st32(tl + kTmO + q * 32, o);
+          }
+          ptx::tmem_st_wait();
+          l_run *= f;
+        }
+        m_run = m_tile;
+      }
+      float sum = 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int c0 = h * 64 + 2 * e;
+          const float s0 = __uint_as_float(a[c0 >> 5][c0 & 31]);
+          const float s1 = __uint_as_float(a[(c0 + 1) >> 5][(c0 + 1) & 31]);
+          const float p0 = c0 < valid_n ? ptx::ex2(fmaf(s0, p.scale_log2, -m_run)) : 0.f;
+          const float p1 = c0 + 1 < valid_n ? ptx::ex2(fmaf(s1, p.scale_log2, -m_run)) : 0.f;
+          sum += p0 + p1;
+          pk[e] = pack_bf16(p0, p1);
+        }
+        ptx::tmem_st32(tl + kTmP + s * 64 + h * 32, pk);
+      }
+      l_run += sum;
+      ptx::tmem_st_wait();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&bars.p_full[s]);
+    }
+    if (ok && !ptx::mbar_wait(&bars.o_final, 0, abort_flag, kWaitNs)) ok = false;
+    if (!ok) {
+      fail(bars, p.status);
+    } else {
+      ptx::tc_fence_after();
+      uint32_t o[4][32];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) ptx::tmem_ld32(tl + kTmO + q * 32, o[q]);
+      ptx::tmem_ld_wait(o[0]);
+      ptx::reg_barrier(o[1]);
+      ptx::reg_barrier(o[2]);
+      ptx::reg_barrier(o[3]);
+      if (tok >= 0) {
+        const float inv = 1.f / l_run;
+        const int64_t row = (bh * p.n_q + tok) * kD;
+#pragma unroll
+        for (int c = 0; c < kD; c += 8) {
+          float v[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(o[(c + e) >> 5][(c + e) & 31]) * inv;
+          if (kAnchor) {
+            float of[8];
+            load8(p.O_full + row + c, of);
+            float4* dst = reinterpret_cast<float4*>(p.R_out + row + c);
+            dst[0] = make_float4(of[0] - v[0], of[1] - v[1], of[2] - v[2], of[3] - v[3]);
+            dst[1] = make_float4(of[4] - v[4], of[5] - v[5], of[6] - v[6], of[7] - v[7]);
+          } else {
+            const float4* rr = reinterpret_cast<const float4*>(p.R_in + row + c);
+            const float4 r0 = rr[0], r1 = rr[1];
+            uint4 out;
+            out.x = pack_bf16(v[0] + r0.x, v[1] + r0.y);
+            out.y = pack_bf16(v[2] + r0.z, v[3] + r0.w);
+            out.z = pack_bf16(v[4] + r1.x, v[5] + r1.y);
+            out.w = pack_bf16(v[6] + r1.z, v[7] + r1.w);
+            *reinterpret_cast<uint4*>(p.O_out + row + c) = out;
+          }
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, kTmCols);
+  }
+}
+
+}  // namespace
+
+bool tc_sparse_supported(const AttnArgs& a) { return a.bf16 && a.d == kD; }
+
+int tc_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices,
+              const void* O_full, float* R_out, const float* R_in, void* O_out,
+              cudaStream_t st) {
+  SparseParams p;
+  p.Q = (const __nv_bfloat16*)a.Q;
+  p.K = (const __nv_bfloat16*)a.K;
+  p.V = (const __nv_bfloat16*)a.V;
+  p.groups = groups;
+  p.indices = indices;
+  p.n_q = a.n_q;
+  p.n_kv = a.n_kv;
+  p.gs = a.gs;
+  p.G = a.G;
+  p.k = a.k;
+  p.tiles_per_group = (a.gs + kTile - 1) / kTile;
+  p.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
+  p.O_full = (const __nv_bfloat16*)O_full;
+  p.R_out = R_out;
+  p.R_in = R_in;
+  p.O_out = (__nv_bfloat16*)O_out;
+  p.status = a.status;
+  const int64_t tiles = a.BH * a.G * p.tiles_per_group;
+  if (tiles > 0x7fffffffLL) return TLSP_ERR_UNSUPPORTED;
+  if (R_out) {
+    cudaFuncSetAttribute(sparse_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)kSmemBytes);
+    sparse_tc_kernel<true><<<(unsigned)tiles, kThreads, kSmemBytes, st>>>(p);
+  } else {
+    cudaFuncSetAttribute(sparse_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)kSmemBytes);
+    sparse_tc_kernel<false><<<(unsigned)tiles, kThreads, kSmemBytes, st>>>(p);
+  }
+  return check_launch();
+}
+
+}  // namespace tlsp

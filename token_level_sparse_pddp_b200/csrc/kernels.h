@@ -39,4 +39,18 @@ int simt_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices
                 const void* O_full, float* R_out, const float* R_in, void* O_out,
                 cudaStream_t st);
 
+// attn_tc_sparse.cu: tensor-core gathered sparse attention (bf16, d = 128)
+bool tc_sparse_supported(const AttnArgs& a);
+int tc_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices,
+              const void* O_full, float* R_out, const float* R_in, void* O_out,
+              cudaStream_t st);
+
+// Sparse pass with the residual epilogue on the best kernel for the shape.
+inline int sparse_pass(const AttnArgs& a, const int32_t* groups, const int32_t* indices,
+                       const void* O_full, float* R_out, const float* R_in, void* O_out,
+                       cudaStream_t st) {
+  if (tc_sparse_supported(a)) return tc_sparse(a, groups, indices, O_full, R_out, R_in, O_out, st);
+  return simt_sparse(a, groups, indices, O_full, R_out, R_in, O_out, st);
+}
+
 }  // namespace tlsp
