@@ -10,16 +10,18 @@
 // tile; the padding rows of a ragged group are zero and never written back).
 // Warp roles:
 //   warps 0-3  softmax + epilogue: thread t owns query row t = TMEM lane t;
-//   warps 4-7  producers: gather the tile's Q rows and, 128 selected keys at
-//              a time, the K and V rows with 16-byte cp.async into 128-byte
-//              swizzled shared memory (the tcgen05 canonical layout);
+//   warps 4-7  producers: together gather the tile's Q rows; then warps 4-5
+//              stream the K rows and warps 6-7 the V rows of the selection,
+//              128 keys at a time, with 16-byte cp.async into 128-byte
+//              swizzled shared memory (the tcgen05 canonical layout); the
+//              indices of the next chunk are loaded while a chunk is in flight;
 //   warp 8     allocates TMEM; lane 0 issues the tcgen05.mma instructions.
 // Per chunk j of 128 keys: S_j = Q K_j^T (M=N=K=128, fp32 in TMEM), online
 // softmax with exp2 on the SFU, P_j (bf16) written back to TMEM, and
 // O += P_j V_j with A read from TMEM and V as an MN-major B operand.
 // TMEM columns: S double buffer [0,256), O [256,384), P double buffer
-// [384,512). K and V have two shared-memory slots each, so the gather of
-// chunk j+2 overlaps the math of chunks j and j+1.
+// [384,512). K has three shared-memory slots and V two, so gathers run
+// ahead of the math by two chunks.
 // The running max is only raised when it grows by more than 2^8 (then O is
 // rescaled in TMEM); between raises the stale max is used for both the
 // numerator and the denominator, which cancels exactly in O / l.
@@ -36,10 +38,11 @@ constexpr int kD = 128;
 constexpr int kThreads = 288;
 constexpr uint32_t kTileBytes = kTile * kD * 2;  // 32 KB
 constexpr uint32_t kHalfBytes = kTileBytes / 2;  // one 64-column half: 128 rows x 128 B
+constexpr int kKSlots = 3, kVSlots = 2;
 constexpr uint32_t kSmQ = 0;
-constexpr uint32_t kSmK = kTileBytes;      // 2 slots
-constexpr uint32_t kSmV = 3 * kTileBytes;  // 2 slots
-constexpr uint32_t kSmBar = 5 * kTileBytes;
+constexpr uint32_t kSmK = kTileBytes;                        // kKSlots slots
+constexpr uint32_t kSmV = (1 + kKSlots) * kTileBytes;        // kVSlots slots
+constexpr uint32_t kSmBar = (1 + kKSlots + kVSlots) * kTileBytes;
 constexpr uint32_t kSmemBytes = kSmBar + 256 + 1024;  // + slack to align the base to 1024 B
 constexpr uint32_t kTmCols = 512;
 constexpr uint32_t kTmS = 0, kTmO = 256, kTmP = 384;
@@ -48,7 +51,7 @@ constexpr float kRescaleLog2 = 8.f;
 
 struct Bars {
   uint64_t q_full;
-  uint64_t k_full[2], v_full[2], k_empty[2], v_empty[2];
+  uint64_t k_full[kKSlots], k_empty[kKSlots], v_full[kVSlots], v_empty[kVSlots];
   uint64_t s_full[2], p_full[2];
   uint64_t o_done, o_final, drain;
   uint32_t tmem_base;
@@ -78,18 +81,38 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
   return (uint32_t)(c >> 3) * kHalfBytes + (uint32_t)r * 128u + ((uint32_t)((c & 7) ^ (r & 7)) << 4);
 }
 
-// 16 copies per producer thread: 128 rows x 16 chunks; consecutive threads
-// take consecutive chunks of a row (two 256-byte rows per warp instruction).
-template <class RowOf>
-__device__ __forceinline__ void gather_tile(uint32_t dst, const __nv_bfloat16* src, RowOf row_of,
-                                            int p) {
-#pragma unroll 4
-  for (int it = 0; it < 16; ++it) {
-    const int lin = it * 128 + p;
-    const int r = lin >> 4, c = lin & 15;
-    const int row = row_of(r);
+// Gathers a [128 x 128] bf16 tile whose row r is global row rows(r) (or
+// zeros for rows(r) < 0) with NT threads; thread pt copies 16-byte chunk
+// c = pt % 16 of rows it * (NT / 16) + pt / 16, so a warp instruction moves
+// two whole 256-byte rows.
+template <int NT>
+__device__ __forceinline__ void gather_rows(uint32_t dst, const __nv_bfloat16* src,
+                                            const int (&rows)[2048 / NT], int pt) {
+  const int c = pt & 15;
+#pragma unroll
+  for (int it = 0; it < 2048 / NT; ++it) {
+    const int r = it * (NT / 16) + (pt >> 4);
+    const int row = rows[it];
     const __nv_bfloat16* s = src + (row >= 0 ? (int64_t)row * kD + c * 8 : 0);
     ptx::cp_async16(dst + swz(r, c), s, row >= 0 ? 16u : 0u);
+  }
+}
+
+// Global rows of chunk j of the selection for a producer thread of NT.
+template <int NT>
+__device__ __forceinline__ void chunk_rows(const int32_t* sel, int j, int k, int n_kv, int pt,
+                                           int (&rows)[2048 / NT], int* status) {
+#pragma unroll
+  for (int it = 0; it < 2048 / NT; ++it) {
+    const int q = j * kTile + it * (NT / 16) + (pt >> 4);
+    rows[it] = q < k ? __ldg(sel + q) : -1;
+  }
+#pragma unroll
+  for (int it = 0; it < 2048 / NT; ++it) {
+    if (rows[it] >= n_kv) {
+      record_status(status, TLSP_ERR_DEVICE_ASSERT);
+      rows[it] = -1;
+    }
   }
 }
 
@@ -123,11 +146,15 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
 
   if (tid == 0) {
     ptx::mbar_init(&bars.q_full, 128);
-    for (int s = 0; s < 2; ++s) {
-      ptx::mbar_init(&bars.k_full[s], 128);
-      ptx::mbar_init(&bars.v_full[s], 128);
+    for (int s = 0; s < kKSlots; ++s) {
+      ptx::mbar_init(&bars.k_full[s], 64);
       ptx::mbar_init(&bars.k_empty[s], 1);
+    }
+    for (int s = 0; s < kVSlots; ++s) {
+      ptx::mbar_init(&bars.v_full[s], 64);
       ptx::mbar_init(&bars.v_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&bars.s_full[s], 1);
       ptx::mbar_init(&bars.p_full[s], 128);
     }
@@ -148,45 +175,44 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
 
   if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ producers
+    // all 128 gather Q; then warps 4-5 stream K chunks and warps 6-7 V chunks
     const int pt = tid - 128;
     const __nv_bfloat16* Qbh = p.Q + bh * (int64_t)p.n_q * kD;
-    const __nv_bfloat16* Kbh = p.K + bh * (int64_t)p.n_kv * kD;
-    const __nv_bfloat16* Vbh = p.V + bh * (int64_t)p.n_kv * kD;
-    gather_tile(base + kSmQ, Qbh, [&](int r) -> int {
-      const int gr = t * kTile + r;
-      if (gr >= p.gs) return -1;
-      const int tok = grp[gr];
-      if (tok >= p.n_q) {
-        record_status(p.status, TLSP_ERR_DEVICE_ASSERT);
-        return -1;
+    {
+      int rows[16];
+#pragma unroll
+      for (int it = 0; it < 16; ++it) {
+        const int gr = t * kTile + it * 8 + (pt >> 4);
+        rows[it] = gr < p.gs ? __ldg(grp + gr) : -1;
       }
-      return tok;
-    }, pt);
-    ptx::cp_async_arrive_noinc(&bars.q_full);
-    for (int j = 0; j < n_chunks; ++j) {
-      const int s = j & 1;
-      auto kv_row = [&](int r) -> int {
-        const int q = j * kTile + r;
-        if (q >= p.k) return -1;
-        const int kv = __ldg(sel + q);
-        if ((unsigned)kv >= (unsigned)p.n_kv) {
+#pragma unroll
+      for (int it = 0; it < 16; ++it) {
+        if (rows[it] >= p.n_q) {
           record_status(p.status, TLSP_ERR_DEVICE_ASSERT);
-          return -1;
+          rows[it] = -1;
         }
-        return kv;
-      };
-      if (j >= 2 && !ptx::mbar_wait(&bars.k_empty[s], ((j >> 1) - 1) & 1, abort_flag, kWaitNs)) {
+      }
+      gather_rows<128>(base + kSmQ, Qbh, rows, pt);
+      ptx::cp_async_arrive_noinc(&bars.q_full);
+    }
+    const bool is_k = warp < 6;
+    const int qt = pt & 63;
+    const __nv_bfloat16* src = (is_k ? p.K : p.V) + bh * (int64_t)p.n_kv * kD;
+    const int nslots = is_k ? kKSlots : kVSlots;
+    const uint32_t slot0 = base + (is_k ? kSmK : kSmV);
+    uint64_t* full = is_k ? bars.k_full : bars.v_full;
+    uint64_t* empty = is_k ? bars.k_empty : bars.v_empty;
+    int rows[32];
+    chunk_rows<64>(sel, 0, p.k, p.n_kv, qt, rows, p.status);
+    for (int j = 0; j < n_chunks; ++j) {
+      const int s = j % nslots, u = j / nslots;
+      if (u > 0 && !ptx::mbar_wait(&empty[s], (u - 1) & 1, abort_flag, kWaitNs)) {
         fail(bars, p.status);
         break;
       }
-      gather_tile(base + kSmK + s * kTileBytes, Kbh, kv_row, pt);
-      ptx::cp_async_arrive_noinc(&bars.k_full[s]);
-      if (j >= 2 && !ptx::mbar_wait(&bars.v_empty[s], ((j >> 1) - 1) & 1, abort_flag, kWaitNs)) {
-        fail(bars, p.status);
-        break;
-      }
-      gather_tile(base + kSmV + s * kTileBytes, Vbh, kv_row, pt);
-      ptx::cp_async_arrive_noinc(&bars.v_full[s]);
+      gather_rows<64>(slot0 + s * kTileBytes, src, rows, qt);
+      ptx::cp_async_arrive_noinc(&full[s]);
+      if (j + 1 < n_chunks) chunk_rows<64>(sel, j + 1, p.k, p.n_kv, qt, rows, p.status);
     }
     ptx::cp_async_wait_all();
   } else if (warp == 8) {
@@ -196,12 +222,12 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
       constexpr uint32_t id_pv = ptx::idesc_bf16(kTile, kD, true);
       bool ok = ptx::mbar_wait(&bars.q_full, 0, abort_flag, kWaitNs);
       auto issue_qk = [&](int j) {
-        const int s = j & 1;
-        ok = ok && ptx::mbar_wait(&bars.k_full[s], (j >> 1) & 1, abort_flag, kWaitNs);
+        const int s = j & 1, ks = j % kKSlots;
+        ok = ok && ptx::mbar_wait(&bars.k_full[ks], (j / kKSlots) & 1, abort_flag, kWaitNs);
         if (!ok) return;
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_after();
-        const uint32_t kb = base + kSmK + s * kTileBytes;
+        const uint32_t kb = base + kSmK + ks * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t off = (uint32_t)(kk >> 2) * kHalfBytes + (uint32_t)(kk & 3) * 32u;
@@ -209,25 +235,25 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
                       ptx::sw128_desc(kb + off, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
         }
         ptx::tc_commit(&bars.s_full[s]);
-        ptx::tc_commit(&bars.k_empty[s]);
+        ptx::tc_commit(&bars.k_empty[ks]);
       };
       issue_qk(0);
       if (n_chunks > 1) issue_qk(1);
       for (int j = 0; j < n_chunks && ok; ++j) {
-        const int s = j & 1;
+        const int s = j & 1, vs = j % kVSlots;
         ok = ptx::mbar_wait(&bars.p_full[s], (j >> 1) & 1, abort_flag, kWaitNs) &&
-             ptx::mbar_wait(&bars.v_full[s], (j >> 1) & 1, abort_flag, kWaitNs);
+             ptx::mbar_wait(&bars.v_full[vs], (j / kVSlots) & 1, abort_flag, kWaitNs);
         if (!ok) break;
         ptx::fence_proxy_async_smem();
         ptx::tc_fence_after();
-        const uint32_t vb = base + kSmV + s * kTileBytes;
+        const uint32_t vb = base + kSmV + vs * kTileBytes;
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk) {
           ptx::mma_ts(tmem + kTmO, tmem + kTmP + s * 64 + kk * 8,
                       ptx::sw128_desc(vb + kk * 2048, kHalfBytes, 1024), id_pv,
                       (j > 0 || kk > 0) ? 1u : 0u);
         }
-        ptx::tc_commit(&bars.v_empty[s]);
+        ptx::tc_commit(&bars.v_empty[vs]);
         ptx::tc_commit(j == n_chunks - 1 ? &bars.o_final : &bars.o_done);
         if (j + 2 < n_chunks) issue_qk(j + 2);
       }
@@ -262,11 +288,18 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
       ptx::reg_barrier(a[3]);
       const int valid_n = min(kTile, p.k - j * kTile);
       float mx = -INFINITY;
+      if (valid_n == kTile) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
+        for (int q = 0; q < 4; ++q)
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (q * 32 + e < valid_n) mx = fmaxf(mx, __uint_as_float(a[q][e]));
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(a[q][e]));
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (q * 32 + e < valid_n) mx = fmaxf(mx, __uint_as_float(a[q][e]));
+      }
       const float m_tile = mx * p.scale_log2;
       if (m_tile > m_run + kRescaleLog2) {
         if (j > 0) {
@@ -292,18 +325,31 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
         m_run = m_tile;
       }
       float sum = 0.f;
+      const float neg_m = -m_run;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
+        if (valid_n == kTile) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int c0 = h * 64 + 2 * e;
-          const float s0 = __uint_as_float(a[c0 >> 5][c0 & 31]);
-          const float s1 = __uint_as_float(a[(c0 + 1) >> 5][(c0 + 1) & 31]);
-          const float p0 = c0 < valid_n ? ptx::ex2(fmaf(s0, p.scale_log2, -m_run)) : 0.f;
-          const float p1 = c0 + 1 < valid_n ? ptx::ex2(fmaf(s1, p.scale_log2, -m_run)) : 0.f;
-          sum += p0 + p1;
-          pk[e] = pack_bf16(p0, p1);
+          for (int e = 0; e < 32; ++e) {
+            const int c0 = h * 64 + 2 * e;
+            const float p0 = ptx::ex2(fmaf(__uint_as_float(a[c0 >> 5][c0 & 31]), p.scale_log2, neg_m));
+            const float p1 =
+                ptx::ex2(fmaf(__uint_as_float(a[(c0 + 1) >> 5][(c0 + 1) & 31]), p.scale_log2, neg_m));
+            sum += p0 + p1;
+            pk[e] = pack_bf16(p0, p1);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int c0 = h * 64 + 2 * e;
+            const float s0 = __uint_as_float(a[c0 >> 5][c0 & 31]);
+            const float s1 = __uint_as_float(a[(c0 + 1) >> 5][(c0 + 1) & 31]);
+            const float p0 = c0 < valid_n ? ptx::ex2(fmaf(s0, p.scale_log2, neg_m)) : 0.f;
+            const float p1 = c0 + 1 < valid_n ? ptx::ex2(fmaf(s1, p.scale_log2, neg_m)) : 0.f;
+            sum += p0 + p1;
+            pk[e] = pack_bf16(p0, p1);
+          }
         }
         ptx::tmem_st32(tl + kTmP + s * 64 + h * 32, pk);
       }
