@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run the workload with only this many heads (smaller case for profiling)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -197,6 +199,9 @@ def main():
     args = parse()
     from token_level_sparse_pddp_b200.synthetic import InputStream, workload
     wl = workload(args.workload)
+    if args.heads:
+        import dataclasses
+        wl = dataclasses.replace(wl, heads=args.heads, name=f"{wl.name}-H{args.heads}")
     if args.impl == "reference":
         os.environ.setdefault("OMP_NUM_THREADS", str(os.cpu_count() or 1))
         reference_arm(args, wl)
