@@ -43,7 +43,9 @@ constexpr uint32_t kSmQ = 0;
 constexpr uint32_t kSmK = kTileBytes;                        // kKSlots slots
 constexpr uint32_t kSmV = (1 + kKSlots) * kTileBytes;        // kVSlots slots
 constexpr uint32_t kSmBar = (1 + kKSlots + kVSlots) * kTileBytes;
-constexpr uint32_t kSmemBytes = kSmBar + 256 + 1024;  // + slack to align the base to 1024 B
+constexpr uint32_t kSmIdx = kSmBar + 256;  // the tile's selection, when it fits
+constexpr int kIdxCap = 8192;
+constexpr uint32_t kSmemBytes = kSmIdx + kIdxCap * 4 + 1024;  // + slack to align the base
 constexpr uint32_t kTmCols = 512;
 constexpr uint32_t kTmS = 0, kTmO = 256, kTmP = 384;
 constexpr uint64_t kWaitNs = 1000000000ull;
@@ -60,17 +62,17 @@ struct Bars {
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
 struct SparseParams {
-  const __nv_bfloat16* Q;
-  const __nv_bfloat16* K;
-  const __nv_bfloat16* V;
-  const int32_t* groups;
-  const int32_t* indices;
+  const __nv_bfloat16* __restrict__ Q;
+  const __nv_bfloat16* __restrict__ K;
+  const __nv_bfloat16* __restrict__ V;
+  const int32_t* __restrict__ groups;
+  const int32_t* __restrict__ indices;
   int n_q, n_kv, gs, G, k, tiles_per_group;
   float scale_log2;
-  const __nv_bfloat16* O_full;
-  float* R_out;
-  const float* R_in;
-  __nv_bfloat16* O_out;
+  const __nv_bfloat16* __restrict__ O_full;
+  float* __restrict__ R_out;
+  const float* __restrict__ R_in;
+  __nv_bfloat16* __restrict__ O_out;
   int* status;
 };
 
@@ -98,14 +100,15 @@ __device__ __forceinline__ void gather_rows(uint32_t dst, const __nv_bfloat16* s
   }
 }
 
-// Global rows of chunk j of the selection for a producer thread of NT.
+// Global rows of chunk j of the selection for a producer thread of NT
+// (sel points at the selection in shared or global memory).
 template <int NT>
 __device__ __forceinline__ void chunk_rows(const int32_t* sel, int j, int k, int n_kv, int pt,
                                            int (&rows)[2048 / NT], int* status) {
 #pragma unroll
   for (int it = 0; it < 2048 / NT; ++it) {
     const int q = j * kTile + it * (NT / 16) + (pt >> 4);
-    rows[it] = q < k ? __ldg(sel + q) : -1;
+    rows[it] = q < k ? sel[q] : -1;
   }
 #pragma unroll
   for (int it = 0; it < 2048 / NT; ++it) {
@@ -195,6 +198,19 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
       gather_rows<128>(base + kSmQ, Qbh, rows, pt);
       ptx::cp_async_arrive_noinc(&bars.q_full);
     }
+    // The tile's selection goes to shared memory once (4-byte cp.async by all
+    // 128 producers), so no chunk waits on an index load.
+    const bool idx_smem = p.k <= kIdxCap;
+    int32_t* sel_s = reinterpret_cast<int32_t*>(smem + kSmIdx);
+    if (idx_smem) {
+      for (int q = pt; q < p.k; q += 128)
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(base + kSmIdx + 4u * q),
+                     "l"(sel + q)
+                     : "memory");
+      ptx::cp_async_wait_all();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+    }
+    const int32_t* selp = idx_smem ? sel_s : sel;
     const bool is_k = warp < 6;
     const int qt = pt & 63;
     const __nv_bfloat16* src = (is_k ? p.K : p.V) + bh * (int64_t)p.n_kv * kD;
@@ -203,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
     uint64_t* full = is_k ? bars.k_full : bars.v_full;
     uint64_t* empty = is_k ? bars.k_empty : bars.v_empty;
     int rows[32];
-    chunk_rows<64>(sel, 0, p.k, p.n_kv, qt, rows, p.status);
+    chunk_rows<64>(selp, 0, p.k, p.n_kv, qt, rows, p.status);
     for (int j = 0; j < n_chunks; ++j) {
       const int s = j % nslots, u = j / nslots;
       if (u > 0 && !ptx::mbar_wait(&empty[s], (u - 1) & 1, abort_flag, kWaitNs)) {
@@ -212,7 +228,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
       }
       gather_rows<64>(slot0 + s * kTileBytes, src, rows, qt);
       ptx::cp_async_arrive_noinc(&full[s]);
-      if (j + 1 < n_chunks) chunk_rows<64>(sel, j + 1, p.k, p.n_kv, qt, rows, p.status);
+      if (j + 1 < n_chunks) chunk_rows<64>(selp, j + 1, p.k, p.n_kv, qt, rows, p.status);
     }
     ptx::cp_async_wait_all();
   } else if (warp == 8) {
@@ -289,10 +305,19 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
       const int valid_n = min(kTile, p.k - j * kTile);
       float mx = -INFINITY;
       if (valid_n == kTile) {
+        // 16 independent partial maxima, then a tree
+        float pm[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pm[e] = -INFINITY;
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(a[q][e]));
+          for (int e = 0; e < 32; ++e) pm[e & 15] = fmaxf(pm[e & 15], __uint_as_float(a[q][e]));
+#pragma unroll
+        for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+          for (int e = 0; e < w; ++e) pm[e] = fmaxf(pm[e], pm[e + w]);
+        mx = pm[0];
       } else {
 #pragma unroll
         for (int q = 0; q < 4; ++q)
@@ -324,7 +349,9 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
         }
         m_run = m_tile;
       }
-      float sum = 0.f;
+      float ps[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ps[e] = 0.f;
       const float neg_m = -m_run;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -336,7 +363,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
             const float p0 = ptx::ex2(fmaf(__uint_as_float(a[c0 >> 5][c0 & 31]), p.scale_log2, neg_m));
             const float p1 =
                 ptx::ex2(fmaf(__uint_as_float(a[(c0 + 1) >> 5][(c0 + 1) & 31]), p.scale_log2, neg_m));
-            sum += p0 + p1;
+            ps[e & 7] += p0 + p1;
             pk[e] = pack_bf16(p0, p1);
           }
         } else {
@@ -347,52 +374,65 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
             const float s1 = __uint_as_float(a[(c0 + 1) >> 5][(c0 + 1) & 31]);
             const float p0 = c0 < valid_n ? ptx::ex2(fmaf(s0, p.scale_log2, neg_m)) : 0.f;
             const float p1 = c0 + 1 < valid_n ? ptx::ex2(fmaf(s1, p.scale_log2, neg_m)) : 0.f;
-            sum += p0 + p1;
+            ps[e & 7] += p0 + p1;
             pk[e] = pack_bf16(p0, p1);
           }
         }
         ptx::tmem_st32(tl + kTmP + s * 64 + h * 32, pk);
       }
-      l_run += sum;
+      l_run += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       ptx::tmem_st_wait();
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bars.p_full[s]);
+    }
+    // The row this thread finishes is pulled towards L1 while the last PV runs.
+    const int64_t row = (bh * p.n_q + (tok >= 0 ? tok : 0)) * kD;
+    if (tok >= 0) {
+      const char* pre = kAnchor ? (const char*)(p.O_full + row) : (const char*)(p.R_in + row);
+      const int lines = kAnchor ? 2 : 4;
+      for (int l = 0; l < lines; ++l)
+        asm volatile("prefetch.global.L1 [%0];" ::"l"(pre + 128 * l));
     }
     if (ok && !ptx::mbar_wait(&bars.o_final, 0, abort_flag, kWaitNs)) ok = false;
     if (!ok) {
       fail(bars, p.status);
     } else {
       ptx::tc_fence_after();
-      uint32_t o[4][32];
+      const float inv = 1.f / l_run;
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        uint32_t o[32];
+        ptx::tmem_ld32(tl + kTmO + q * 32, o);
+        ptx::tmem_ld_wait(o);
+        if (tok < 0) continue;
+        const int c0 = q * 32;
+        if (kAnchor) {
+          float of[32];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) ptx::tmem_ld32(tl + kTmO + q * 32, o[q]);
-      ptx::tmem_ld_wait(o[0]);
-      ptx::reg_barrier(o[1]);
-      ptx::reg_barrier(o[2]);
-      ptx::reg_barrier(o[3]);
-      if (tok >= 0) {
-        const float inv = 1.f / l_run;
-        const int64_t row = (bh * p.n_q + tok) * kD;
+          for (int c = 0; c < 32; c += 8) load8(p.O_full + row + c0 + c, of + c);
+          float4* dst = reinterpret_cast<float4*>(p.R_out + row + c0);
 #pragma unroll
-        for (int c = 0; c < kD; c += 8) {
-          float v[8];
+          for (int c = 0; c < 32; c += 4)
+            dst[c / 4] = make_float4(of[c] - __uint_as_float(o[c]) * inv,
+                                     of[c + 1] - __uint_as_float(o[c + 1]) * inv,
+                                     of[c + 2] - __uint_as_float(o[c + 2]) * inv,
+                                     of[c + 3] - __uint_as_float(o[c + 3]) * inv);
+        } else {
+          float4 rr[8];
+          const float4* rs = reinterpret_cast<const float4*>(p.R_in + row + c0);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(o[(c + e) >> 5][(c + e) & 31]) * inv;
-          if (kAnchor) {
-            float of[8];
-            load8(p.O_full + row + c, of);
-            float4* dst = reinterpret_cast<float4*>(p.R_out + row + c);
-            dst[0] = make_float4(of[0] - v[0], of[1] - v[1], of[2] - v[2], of[3] - v[3]);
-            dst[1] = make_float4(of[4] - v[4], of[5] - v[5], of[6] - v[6], of[7] - v[7]);
-          } else {
-            const float4* rr = reinterpret_cast<const float4*>(p.R_in + row + c);
-            const float4 r0 = rr[0], r1 = rr[1];
+          for (int c = 0; c < 8; ++c) rr[c] = rs[c];
+          uint4* dst = reinterpret_cast<uint4*>(p.O_out + row + c0);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const float4 r0 = rr[2 * c], r1 = rr[2 * c + 1];
+            const float* v = reinterpret_cast<const float*>(o) + 8 * c;
             uint4 out;
-            out.x = pack_bf16(v[0] + r0.x, v[1] + r0.y);
-            out.y = pack_bf16(v[2] + r0.z, v[3] + r0.w);
-            out.z = pack_bf16(v[4] + r1.x, v[5] + r1.y);
-            out.w = pack_bf16(v[6] + r1.z, v[7] + r1.w);
-            *reinterpret_cast<uint4*>(p.O_out + row + c) = out;
+            out.x = pack_bf16(v[0] * inv + r0.x, v[1] * inv + r0.y);
+            out.y = pack_bf16(v[2] * inv + r0.z, v[3] * inv + r0.w);
+            out.z = pack_bf16(v[4] * inv + r1.x, v[5] * inv + r1.y);
+            out.w = pack_bf16(v[6] * inv + r1.z, v[7] * inv + r1.w);
+            dst[c] = out;
           }
         }
       }

@@ -1,6 +1,8 @@
 // Internal interface between the C-ABI layer (api.cu) and the kernel files.
 #pragma once
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace tlsp {
@@ -38,6 +40,10 @@ int simt_scores(const AttnArgs& a, const int32_t* groups, const float* LSE, floa
 int simt_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices,
                 const void* O_full, float* R_out, const float* R_in, void* O_out,
                 cudaStream_t st);
+
+// tmap.cu: 2-D bf16 row-major tensor map [rows, cols], 128-byte swizzle
+int make_tmap_bf16_rows(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols,
+                        uint32_t box_cols, uint32_t box_rows);
 
 // attn_tc_sparse.cu: tensor-core gathered sparse attention (bf16, d = 128)
 bool tc_sparse_supported(const AttnArgs& a);

@@ -43,8 +43,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase of `bar` with the given parity to complete. Gives up
-// (returns false) when *abort becomes non-zero or after `limit_ns`; the
-// caller then records the error and unwinds.
+// (returns false) when *abort (if given) becomes non-zero or after
+// `limit_ns`; the caller then records the error and unwinds.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -52,10 +52,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
-      if (*abort) return false;
+      if (abort && *abort) return false;
       if (globaltimer_ns() - t0 > limit_ns) return false;
     }
   }
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// ------------------------------------------------------------------ TMA
+
+// Four rows r0..r3 x one box of columns starting at col of a 2-D tensor map
+// (box one row high) into four consecutive box rows at dst; completion is
+// counted in bytes on bar. Rows outside the tensor are filled with zeros.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, int col, int r0,
+                                            int r1, int r2, int r3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
+      "r"(smem_u32(bar))
+      : "memory");
 }
 
 // ------------------------------------------------------------------ cp.async
