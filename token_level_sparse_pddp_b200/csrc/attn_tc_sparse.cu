@@ -30,6 +30,9 @@
 #include "kernels.h"
 #include "tc_ptx.cuh"
 
+#include <algorithm>
+#include <cstdlib>
+
 namespace tlsp {
 namespace {
 
@@ -178,59 +181,65 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
 
   if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ producers
-    // all 128 gather Q; then warps 4-5 stream K chunks and warps 6-7 V chunks
     const int pt = tid - 128;
-    const __nv_bfloat16* Qbh = p.Q + bh * (int64_t)p.n_q * kD;
-    {
-      int rows[16];
-#pragma unroll
-      for (int it = 0; it < 16; ++it) {
-        const int gr = t * kTile + it * 8 + (pt >> 4);
-        rows[it] = gr < p.gs ? __ldg(grp + gr) : -1;
-      }
-#pragma unroll
-      for (int it = 0; it < 16; ++it) {
-        if (rows[it] >= p.n_q) {
-          record_status(p.status, TLSP_ERR_DEVICE_ASSERT);
-          rows[it] = -1;
-        }
-      }
-      gather_rows<128>(base + kSmQ, Qbh, rows, pt);
-      ptx::cp_async_arrive_noinc(&bars.q_full);
-    }
     // The tile's selection goes to shared memory once (4-byte cp.async by all
-    // 128 producers), so no chunk waits on an index load.
+    // 128 producers, its own commit group), so no chunk waits on an index load.
     const bool idx_smem = p.k <= kIdxCap;
-    int32_t* sel_s = reinterpret_cast<int32_t*>(smem + kSmIdx);
     if (idx_smem) {
       for (int q = pt; q < p.k; q += 128)
         asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(base + kSmIdx + 4u * q),
                      "l"(sel + q)
                      : "memory");
-      ptx::cp_async_wait_all();
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      asm volatile("cp.async.commit_group;" ::: "memory");
     }
-    const int32_t* selp = idx_smem ? sel_s : sel;
-    const bool is_k = warp < 6;
-    const int qt = pt & 63;
-    const __nv_bfloat16* src = (is_k ? p.K : p.V) + bh * (int64_t)p.n_kv * kD;
-    const int nslots = is_k ? kKSlots : kVSlots;
-    const uint32_t slot0 = base + (is_k ? kSmK : kSmV);
-    uint64_t* full = is_k ? bars.k_full : bars.v_full;
-    uint64_t* empty = is_k ? bars.k_empty : bars.v_empty;
-    int rows[32];
-    chunk_rows<64>(selp, 0, p.k, p.n_kv, qt, rows, p.status);
-    for (int j = 0; j < n_chunks; ++j) {
-      const int s = j % nslots, u = j / nslots;
-      if (u > 0 && !ptx::mbar_wait(&empty[s], (u - 1) & 1, abort_flag, kWaitNs)) {
-        fail(bars, p.status);
-        break;
+    const int32_t* selp = idx_smem ? reinterpret_cast<const int32_t*>(smem + kSmIdx) : sel;
+    {
+      // all 128 gather Q; then warps 4-5 stream K chunks and warps 6-7 V chunks
+      const __nv_bfloat16* Qbh = p.Q + bh * (int64_t)p.n_q * kD;
+      {
+        int rows[16];
+#pragma unroll
+        for (int it = 0; it < 16; ++it) {
+          const int gr = t * kTile + it * 8 + (pt >> 4);
+          rows[it] = gr < p.gs ? __ldg(grp + gr) : -1;
+        }
+#pragma unroll
+        for (int it = 0; it < 16; ++it) {
+          if (rows[it] >= p.n_q) {
+            record_status(p.status, TLSP_ERR_DEVICE_ASSERT);
+            rows[it] = -1;
+          }
+        }
+        gather_rows<128>(base + kSmQ, Qbh, rows, pt);
+        ptx::cp_async_arrive_noinc(&bars.q_full);
       }
-      gather_rows<64>(slot0 + s * kTileBytes, src, rows, qt);
-      ptx::cp_async_arrive_noinc(&full[s]);
-      if (j + 1 < n_chunks) chunk_rows<64>(selp, j + 1, p.k, p.n_kv, qt, rows, p.status);
+      if (idx_smem) {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+      }
+      {
+      const bool is_k = warp < 6;
+      const int qt = pt & 63;
+      const __nv_bfloat16* src = (is_k ? p.K : p.V) + bh * (int64_t)p.n_kv * kD;
+      const int nslots = is_k ? kKSlots : kVSlots;
+      const uint32_t slot0 = base + (is_k ? kSmK : kSmV);
+      uint64_t* full = is_k ? bars.k_full : bars.v_full;
+      uint64_t* empty = is_k ? bars.k_empty : bars.v_empty;
+      int rows[32];
+      chunk_rows<64>(selp, 0, p.k, p.n_kv, qt, rows, p.status);
+      for (int j = 0; j < n_chunks; ++j) {
+        const int s = j % nslots, u = j / nslots;
+        if (u > 0 && !ptx::mbar_wait(&empty[s], (u - 1) & 1, abort_flag, kWaitNs)) {
+          fail(bars, p.status);
+          break;
+        }
+        gather_rows<64>(slot0 + s * kTileBytes, src, rows, qt);
+        ptx::cp_async_arrive_noinc(&full[s]);
+        if (j + 1 < n_chunks) chunk_rows<64>(selp, j + 1, p.k, p.n_kv, qt, rows, p.status);
+      }
+      }
+      ptx::cp_async_wait_all();
     }
-    ptx::cp_async_wait_all();
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -295,38 +304,76 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
         break;
       }
       ptx::tc_fence_after();
-      uint32_t a[4][32];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) ptx::tmem_ld32(tl + kTmS + s * kTile + q * 32, a[q]);
-      ptx::tmem_ld_wait(a[0]);
-      ptx::reg_barrier(a[1]);
-      ptx::reg_barrier(a[2]);
-      ptx::reg_barrier(a[3]);
       const int valid_n = min(kTile, p.k - j * kTile);
-      float mx = -INFINITY;
-      if (valid_n == kTile) {
-        // 16 independent partial maxima, then a tree
-        float pm[16];
+      const uint32_t s_col = tl + kTmS + s * kTile, p_col = tl + kTmP + s * 64;
+      // One pass over the chunk in 32-column blocks (the next block's TMEM load
+      // in flight while a block is processed): P = 2^(s * scale - m_ref) with
+      // the current reference max, packed to bf16 pairs, while the chunk's
+      // true max is tracked. Returns (sum of P, chunk max).
+      auto p_pass = [&](float m_ref, float& sum_out, float& max_out) {
+        const float neg_m = -m_ref;
+        float sm[4] = {0.f, 0.f, 0.f, 0.f}, mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        uint32_t cur[32], nxt[32];
+        ptx::tmem_ld32(s_col, cur);
+        ptx::tmem_ld_wait(cur);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) pm[e] = -INFINITY;
+        for (int b = 0; b < 4; ++b) {
+          if (b < 3) ptx::tmem_ld32(s_col + 32 * (b + 1), nxt);
+          uint32_t pk[16];
+          if (32 * b + 32 <= valid_n) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
+            for (int e = 0; e < 16; ++e) {
+              const float s0 = __uint_as_float(cur[2 * e]), s1 = __uint_as_float(cur[2 * e + 1]);
+              mx[e & 3] = fmaxf(mx[e & 3], fmaxf(s0, s1));
+              const float p0 = ptx::ex2(fmaf(s0, p.scale_log2, neg_m));
+              const float p1 = ptx::ex2(fmaf(s1, p.scale_log2, neg_m));
+              sm[e & 3] += p0 + p1;
+              pk[e] = pack_bf16(p0, p1);
+            }
+          } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) pm[e & 15] = fmaxf(pm[e & 15], __uint_as_float(a[q][e]));
+            for (int e = 0; e < 16; ++e) {
+              const int c0 = 32 * b + 2 * e;
+              const float s0 = c0 < valid_n ? __uint_as_float(cur[2 * e]) : -INFINITY;
+              const float s1 = c0 + 1 < valid_n ? __uint_as_float(cur[2 * e + 1]) : -INFINITY;
+              mx[e & 3] = fmaxf(mx[e & 3], fmaxf(s0, s1));
+              const float p0 = c0 < valid_n ? ptx::ex2(fmaf(s0, p.scale_log2, neg_m)) : 0.f;
+              const float p1 = c0 + 1 < valid_n ? ptx::ex2(fmaf(s1, p.scale_log2, neg_m)) : 0.f;
+              sm[e & 3] += p0 + p1;
+              pk[e] = pack_bf16(p0, p1);
+            }
+          }
+          ptx::tmem_st16(p_col + 16 * b, pk);
+          if (b < 3) {
+            ptx::tmem_ld_wait(nxt);
 #pragma unroll
-        for (int w = 8; w > 0; w >>= 1)
-#pragma unroll
-          for (int e = 0; e < w; ++e) pm[e] = fmaxf(pm[e], pm[e + w]);
-        mx = pm[0];
+            for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
+          }
+        }
+        sum_out = (sm[0] + sm[1]) + (sm[2] + sm[3]);
+        max_out = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      };
+      float sum, mx;
+      bool raise = (j == 0);
+      if (!raise) {
+        p_pass(m_run, sum, mx);  // speculative: usually the reference max still holds
+        raise = mx * p.scale_log2 > m_run + kRescaleLog2;
       } else {
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
+        // first chunk: its max becomes the reference
+        float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll 1
+        for (int b = 0; b < 4; ++b) {
+          uint32_t c[32];
+          ptx::tmem_ld32(s_col + 32 * b, c);
+          ptx::tmem_ld_wait(c);
 #pragma unroll
           for (int e = 0; e < 32; ++e)
-            if (q * 32 + e < valid_n) mx = fmaxf(mx, __uint_as_float(a[q][e]));
+            if (32 * b + e < valid_n) pm[e & 3] = fmaxf(pm[e & 3], __uint_as_float(c[e]));
+        }
+        mx = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
       }
-      const float m_tile = mx * p.scale_log2;
-      if (m_tile > m_run + kRescaleLog2) {
+      if (raise) {
+        const float m_tile = mx * p.scale_log2;
         if (j > 0) {
           // raise the reference max: O *= 2^(m_run - m_tile) once PV(j-1) has landed
           const float f = ptx::ex2(m_run - m_tile);
@@ -344,43 +391,13 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
             ptx::tmem_st32(tl + kTmO + q * 32, o);
           }
-          ptx::tmem_st_wait();
           l_run *= f;
         }
         m_run = m_tile;
+        ptx::tmem_st_wait();
+        p_pass(m_run, sum, mx);
       }
-      float ps[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) ps[e] = 0.f;
-      const float neg_m = -m_run;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
-        if (valid_n == kTile) {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int c0 = h * 64 + 2 * e;
-            const float p0 = ptx::ex2(fmaf(__uint_as_float(a[c0 >> 5][c0 & 31]), p.scale_log2, neg_m));
-            const float p1 =
-                ptx::ex2(fmaf(__uint_as_float(a[(c0 + 1) >> 5][(c0 + 1) & 31]), p.scale_log2, neg_m));
-            ps[e & 7] += p0 + p1;
-            pk[e] = pack_bf16(p0, p1);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int c0 = h * 64 + 2 * e;
-            const float s0 = __uint_as_float(a[c0 >> 5][c0 & 31]);
-            const float s1 = __uint_as_float(a[(c0 + 1) >> 5][(c0 + 1) & 31]);
-            const float p0 = c0 < valid_n ? ptx::ex2(fmaf(s0, p.scale_log2, neg_m)) : 0.f;
-            const float p1 = c0 + 1 < valid_n ? ptx::ex2(fmaf(s1, p.scale_log2, neg_m)) : 0.f;
-            ps[e & 7] += p0 + p1;
-            pk[e] = pack_bf16(p0, p1);
-          }
-        }
-        ptx::tmem_st32(tl + kTmP + s * 64 + h * 32, pk);
-      }
-      l_run += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      l_run += sum;
       ptx::tmem_st_wait();
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bars.p_full[s]);
@@ -451,6 +468,13 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
 
 bool tc_sparse_supported(const AttnArgs& a) { return a.bf16 && a.d == kD; }
 
+template <bool kAnchor>
+static void launch_sparse(const SparseParams& p, int64_t tiles, cudaStream_t st) {
+  cudaFuncSetAttribute(sparse_tc_kernel<kAnchor>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)kSmemBytes);
+  sparse_tc_kernel<kAnchor><<<(unsigned)tiles, kThreads, kSmemBytes, st>>>(p);
+}
+
 int tc_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices,
               const void* O_full, float* R_out, const float* R_in, void* O_out,
               cudaStream_t st) {
@@ -474,15 +498,10 @@ int tc_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices,
   p.status = a.status;
   const int64_t tiles = a.BH * a.G * p.tiles_per_group;
   if (tiles > 0x7fffffffLL) return TLSP_ERR_UNSUPPORTED;
-  if (R_out) {
-    cudaFuncSetAttribute(sparse_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)kSmemBytes);
-    sparse_tc_kernel<true><<<(unsigned)tiles, kThreads, kSmemBytes, st>>>(p);
-  } else {
-    cudaFuncSetAttribute(sparse_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)kSmemBytes);
-    sparse_tc_kernel<false><<<(unsigned)tiles, kThreads, kSmemBytes, st>>>(p);
-  }
+  if (R_out)
+    launch_sparse<true>(p, tiles, st);
+  else
+    launch_sparse<false>(p, tiles, st);
   return check_launch();
 }
 
