@@ -189,8 +189,8 @@ int tlsp_anchor_attention(const tlsp_dims* dims, const void* Q, const void* K, c
   const AttnArgs a = attn_args(dims, Q, K, V, group_size, k, ws);
   float* lse = at<float>(ws, L.lse);
   float* S = scores ? scores : at<float>(ws, L.scores);
-  TLSP_TRY(simt_dense(a, O, lse, st));
-  TLSP_TRY(simt_scores(a, groups, lse, S, st));
+  TLSP_TRY(dense_pass(a, O, lse, st));
+  TLSP_TRY(scores_pass(a, groups, lse, S, st));
   TLSP_TRY(launch_topk(S, a.BH * a.G, a.n_kv, k, indices, st));
   return sparse_pass(a, groups, indices, O, R, nullptr, nullptr, st);
 }
@@ -204,7 +204,7 @@ int tlsp_dense_attention(const tlsp_dims* dims, const void* Q, const void* K, co
   const size_t lse_bytes = sizeof(float) * (size_t)dims->batch * dims->heads * dims->n_q;
   if (ws_bytes < kStatusBytes + (lse ? 0 : lse_bytes)) return TLSP_ERR_WORKSPACE;
   const AttnArgs a = attn_args(dims, Q, K, V, 1, 1, ws);
-  return simt_dense(a, O, lse ? lse : at<float>(ws, kStatusBytes), (cudaStream_t)stream);
+  return dense_pass(a, O, lse ? lse : at<float>(ws, kStatusBytes), (cudaStream_t)stream);
 }
 
 int tlsp_reuse_attention(const tlsp_dims* dims, const void* Q, const void* K, const void* V,

@@ -1,40 +1,46 @@
-// Gathered sparse attention on the sm_100a tensor cores (bf16, head_dim 128),
-// with the dense-sparse residual fused into the epilogue.
+// Attention on the sm_100a tensor cores (bf16, head_dim 128): the dense pass
+// of the anchor step and the gathered sparse pass of anchor and reuse steps,
+// with the dense-sparse residual fused into the sparse epilogue.
 //
-// MC-Sparse review, section 3: each query group attends only to its own
-// selected KV tokens (token level, beyond block boundaries). On the anchor
-// step the epilogue stores R = O_full - O_sparse; on reuse steps it returns
-// O_sparse + R (additive correction for the discarded tail).
+// MC-Sparse review, section 3: the anchor step runs dense attention (its
+// output and the exact scores), each query group attends only to its own
+// selected KV tokens (token level, beyond block boundaries), the anchor step
+// stores R = O_full - O_sparse and the reuse steps return O_sparse + R
+// (additive correction for the discarded tail).
 //
-// One CTA per 128-query tile of a group (a group of g_s <= 128 queries is one
-// tile; the padding rows of a ragged group are zero and never written back).
-// Warp roles:
+// One CTA per 128-query tile: a block of 128 consecutive queries (dense) or
+// a group's queries (sparse; g_s <= 128 is one tile, padding rows are zero and
+// never written back). Warp roles (288 threads, one CTA per SM):
 //   warps 0-3  softmax + epilogue: thread t owns query row t = TMEM lane t;
-//   warps 4-7  producers: together gather the tile's Q rows; then warps 4-5
-//              stream the K rows and warps 6-7 the V rows of the selection,
-//              128 keys at a time, with 16-byte cp.async into 128-byte
-//              swizzled shared memory (the tcgen05 canonical layout); the
-//              indices of the next chunk are loaded while a chunk is in flight;
+//   warps 4-7  producers. Dense: lane 0 of warp 4 loads the Q tile and the K
+//              and V tiles of each chunk of 128 keys with TMA box loads.
+//              Sparse: together they load the tile's selection into shared
+//              memory and gather its Q rows, then warps 4-5 gather the K rows
+//              and warps 6-7 the V rows of each chunk of 128 selected keys,
+//              with 16-byte cp.async. Either way the tiles land in 128-byte
+//              swizzled shared memory (the tcgen05 canonical layout);
 //   warp 8     allocates TMEM; lane 0 issues the tcgen05.mma instructions.
-// Per chunk j of 128 keys: S_j = Q K_j^T (M=N=K=128, fp32 in TMEM), online
-// softmax with exp2 on the SFU, P_j (bf16) written back to TMEM, and
-// O += P_j V_j with A read from TMEM and V as an MN-major B operand.
-// TMEM columns: S double buffer [0,256), O [256,384), P double buffer
-// [384,512). K has three shared-memory slots and V two, so gathers run
-// ahead of the math by two chunks.
-// The running max is only raised when it grows by more than 2^8 (then O is
-// rescaled in TMEM); between raises the stale max is used for both the
-// numerator and the denominator, which cancels exactly in O / l.
+// Per chunk j: S_j = Q K_j^T (M=N=K=128, fp32 in TMEM), online softmax with
+// exp2 on the SFU, P_j (bf16) written back to TMEM, and O += P_j V_j with A
+// read from TMEM and V as an MN-major B operand. TMEM columns: S double
+// buffer [0,256), O [256,384), P double buffer [384,512). K has three
+// shared-memory slots and V two, so loads run ahead of the math.
+// The softmax keeps a reference max per row and computes each chunk in one
+// pass against it; only when a chunk's max exceeds the reference by more than
+// 2^8 is the reference raised, O rescaled in TMEM and the chunk recomputed.
+// Between raises the stale reference is used for numerator and denominator
+// alike, which cancels exactly in O / l.
 // Every wait is bounded (1 s); on expiry the kernel records
 // TLSP_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
+#include <algorithm>
+
 #include "kernels.h"
 #include "tc_ptx.cuh"
 
-#include <algorithm>
-#include <cstdlib>
-
 namespace tlsp {
 namespace {
+
+enum Mode { kDense = 0, kAnchor = 1, kReuse = 2 };
 
 constexpr int kTile = 128;
 constexpr int kD = 128;
@@ -43,8 +49,8 @@ constexpr uint32_t kTileBytes = kTile * kD * 2;  // 32 KB
 constexpr uint32_t kHalfBytes = kTileBytes / 2;  // one 64-column half: 128 rows x 128 B
 constexpr int kKSlots = 3, kVSlots = 2;
 constexpr uint32_t kSmQ = 0;
-constexpr uint32_t kSmK = kTileBytes;                        // kKSlots slots
-constexpr uint32_t kSmV = (1 + kKSlots) * kTileBytes;        // kVSlots slots
+constexpr uint32_t kSmK = kTileBytes;                  // kKSlots slots
+constexpr uint32_t kSmV = (1 + kKSlots) * kTileBytes;  // kVSlots slots
 constexpr uint32_t kSmBar = (1 + kKSlots + kVSlots) * kTileBytes;
 constexpr uint32_t kSmIdx = kSmBar + 256;  // the tile's selection, when it fits
 constexpr int kIdxCap = 8192;
@@ -64,18 +70,20 @@ struct Bars {
 };
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
-struct SparseParams {
+struct AttnParams {
+  CUtensorMap tmQ, tmK, tmV;  // dense: [BH*n, 128] bf16 row maps, box 64 x 128, 128-byte swizzle
   const __nv_bfloat16* __restrict__ Q;
   const __nv_bfloat16* __restrict__ K;
   const __nv_bfloat16* __restrict__ V;
   const int32_t* __restrict__ groups;
   const int32_t* __restrict__ indices;
-  int n_q, n_kv, gs, G, k, tiles_per_group;
+  int n_q, n_kv, gs, G, k, tiles_per_group, q_tiles;
   float scale_log2;
-  const __nv_bfloat16* __restrict__ O_full;
-  float* __restrict__ R_out;
-  const float* __restrict__ R_in;
-  __nv_bfloat16* __restrict__ O_out;
+  const __nv_bfloat16* __restrict__ O_full;  // anchor: the dense output as stored
+  float* __restrict__ R_out;                 // anchor
+  const float* __restrict__ R_in;            // reuse
+  __nv_bfloat16* __restrict__ O_out;         // dense and reuse
+  float* __restrict__ lse;                   // dense: [BH, n_q] natural-log partition
   int* status;
 };
 
@@ -132,8 +140,10 @@ __device__ __forceinline__ void fail(Bars& b, int* status) {
   record_status(status, TLSP_ERR_TIMEOUT);
 }
 
-template <bool kAnchor>
-__global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparseParams p) {
+template <int kMode>
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(const __grid_constant__ AttnParams p) {
+  constexpr bool kSparse = kMode != kDense;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -142,22 +152,26 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
   volatile int* abort_flag = &bars.abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int tiles_per_head = p.G * p.tiles_per_group;
+  // tile -> (head, rows): sparse tiles are (group, 128-row part of the group),
+  // dense tiles are blocks of 128 consecutive queries
+  const int tiles_per_head = kSparse ? p.G * p.tiles_per_group : p.q_tiles;
   const int64_t bh = blockIdx.x / tiles_per_head;
   const int rem = blockIdx.x % tiles_per_head;
-  const int g = rem / p.tiles_per_group, t = rem % p.tiles_per_group;
-  const int32_t* grp = p.groups + (bh * p.G + g) * (int64_t)p.gs;
-  const int32_t* sel = p.indices + (bh * p.G + g) * (int64_t)p.k;
-  const int n_chunks = (p.k + kTile - 1) / kTile;
+  const int g = kSparse ? rem / p.tiles_per_group : 0;
+  const int t = kSparse ? rem % p.tiles_per_group : rem;
+  const int32_t* grp = kSparse ? p.groups + (bh * p.G + g) * (int64_t)p.gs : nullptr;
+  const int32_t* sel = kSparse ? p.indices + (bh * p.G + g) * (int64_t)p.k : nullptr;
+  const int n_keys = kSparse ? p.k : p.n_kv;
+  const int n_chunks = (n_keys + kTile - 1) / kTile;
 
   if (tid == 0) {
-    ptx::mbar_init(&bars.q_full, 128);
+    ptx::mbar_init(&bars.q_full, kSparse ? 128 : 1);
     for (int s = 0; s < kKSlots; ++s) {
-      ptx::mbar_init(&bars.k_full[s], 64);
+      ptx::mbar_init(&bars.k_full[s], kSparse ? 64 : 1);
       ptx::mbar_init(&bars.k_empty[s], 1);
     }
     for (int s = 0; s < kVSlots; ++s) {
-      ptx::mbar_init(&bars.v_full[s], 64);
+      ptx::mbar_init(&bars.v_full[s], kSparse ? 64 : 1);
       ptx::mbar_init(&bars.v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -179,7 +193,49 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
   ptx::tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
 
-  if (warp >= 4 && warp < 8) {
+  if (!kSparse && warp == 4) {
+    // ------------------------------------------------------------ dense producer
+    if (lane == 0) {
+      const int q_row = (int)(bh * p.n_q) + t * kTile, kv_row = (int)(bh * p.n_kv);
+      ptx::mbar_arrive_expect_tx(&bars.q_full, kTileBytes);
+      ptx::tma_load_2d(base + kSmQ, &p.tmQ, 0, q_row, &bars.q_full);
+      ptx::tma_load_2d(base + kSmQ + kHalfBytes, &p.tmQ, 64, q_row, &bars.q_full);
+      int issued_k = 0, issued_v = 0;
+      bool ok = true;
+      for (int j = 0; j < n_chunks; ++j) {
+        const int ks = j % kKSlots, ku = j / kKSlots, vs = j % kVSlots, vu = j / kVSlots;
+        const int y = kv_row + j * kTile;
+        if (ku > 0 && !ptx::mbar_wait(&bars.k_empty[ks], (ku - 1) & 1, abort_flag, kWaitNs)) {
+          ok = false;
+          break;
+        }
+        ptx::mbar_arrive_expect_tx(&bars.k_full[ks], kTileBytes);
+        ptx::tma_load_2d(base + kSmK + ks * kTileBytes, &p.tmK, 0, y, &bars.k_full[ks]);
+        ptx::tma_load_2d(base + kSmK + ks * kTileBytes + kHalfBytes, &p.tmK, 64, y,
+                         &bars.k_full[ks]);
+        issued_k = j + 1;
+        if (vu > 0 && !ptx::mbar_wait(&bars.v_empty[vs], (vu - 1) & 1, abort_flag, kWaitNs)) {
+          ok = false;
+          break;
+        }
+        ptx::mbar_arrive_expect_tx(&bars.v_full[vs], kTileBytes);
+        ptx::tma_load_2d(base + kSmV + vs * kTileBytes, &p.tmV, 0, y, &bars.v_full[vs]);
+        ptx::tma_load_2d(base + kSmV + vs * kTileBytes + kHalfBytes, &p.tmV, 64, y,
+                         &bars.v_full[vs]);
+        issued_v = j + 1;
+      }
+      if (!ok) {
+        fail(bars, p.status);
+        // loads already issued land before the CTA's shared memory goes away
+        for (int j = max(0, issued_k - kKSlots); j < issued_k; ++j)
+          ptx::mbar_wait(&bars.k_full[j % kKSlots], (j / kKSlots) & 1, nullptr, kWaitNs);
+        for (int j = max(0, issued_v - kVSlots); j < issued_v; ++j)
+          ptx::mbar_wait(&bars.v_full[j % kVSlots], (j / kVSlots) & 1, nullptr, kWaitNs);
+        ptx::mbar_wait(&bars.q_full, 0, nullptr, kWaitNs);
+      }
+    }
+    __syncwarp();
+  } else if (kSparse && warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ producers
     const int pt = tid - 128;
     // The tile's selection goes to shared memory once (4-byte cp.async by all
@@ -288,13 +344,18 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
       ptx::mbar_wait(&bars.drain, 0, abort_flag, kWaitNs);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 4) {
     // ------------------------------------------------------------ softmax
     const int r = tid;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    const int gr = t * kTile + r;
-    int tok = gr < p.gs ? grp[gr] : -1;
-    if (tok >= p.n_q) tok = -1;
+    int tok;
+    if (kSparse) {
+      const int gr = t * kTile + r;
+      tok = gr < p.gs ? grp[gr] : -1;
+      if (tok >= p.n_q) tok = -1;
+    } else {
+      tok = t * kTile + r < p.n_q ? t * kTile + r : -1;
+    }
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     for (int j = 0; j < n_chunks; ++j) {
@@ -304,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
         break;
       }
       ptx::tc_fence_after();
-      const int valid_n = min(kTile, p.k - j * kTile);
+      const int valid_n = min(kTile, n_keys - j * kTile);
       const uint32_t s_col = tl + kTmS + s * kTile, p_col = tl + kTmP + s * 64;
       // One pass over the chunk in 32-column blocks (the next block's TMEM load
       // in flight while a block is processed): P = 2^(s * scale - m_ref) with
@@ -404,11 +465,10 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
     }
     // The row this thread finishes is pulled towards L1 while the last PV runs.
     const int64_t row = (bh * p.n_q + (tok >= 0 ? tok : 0)) * kD;
-    if (tok >= 0) {
-      const char* pre = kAnchor ? (const char*)(p.O_full + row) : (const char*)(p.R_in + row);
-      const int lines = kAnchor ? 2 : 4;
-      for (int l = 0; l < lines; ++l)
-        asm volatile("prefetch.global.L1 [%0];" ::"l"(pre + 128 * l));
+    if (kMode != kDense && tok >= 0) {
+      const char* pre = kMode == kAnchor ? (const char*)(p.O_full + row) : (const char*)(p.R_in + row);
+      const int lines = kMode == kAnchor ? 2 : 4;
+      for (int l = 0; l < lines; ++l) asm volatile("prefetch.global.L1 [%0];" ::"l"(pre + 128 * l));
     }
     if (ok && !ptx::mbar_wait(&bars.o_final, 0, abort_flag, kWaitNs)) ok = false;
     if (!ok) {
@@ -416,6 +476,8 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
     } else {
       ptx::tc_fence_after();
       const float inv = 1.f / l_run;
+      if (kMode == kDense && tok >= 0)  // log partition in natural units: (m + log2 l) ln 2
+        p.lse[bh * p.n_q + tok] = (m_run + __log2f(l_run)) * 0.6931471805599453f;
 #pragma unroll 1
       for (int q = 0; q < 4; ++q) {
         uint32_t o[32];
@@ -423,7 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
         ptx::tmem_ld_wait(o);
         if (tok < 0) continue;
         const int c0 = q * 32;
-        if (kAnchor) {
+        if (kMode == kAnchor) {
           float of[32];
 #pragma unroll
           for (int c = 0; c < 32; c += 8) load8(p.O_full + row + c0 + c, of + c);
@@ -436,19 +498,27 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
                                      of[c + 3] - __uint_as_float(o[c + 3]) * inv);
         } else {
           float4 rr[8];
-          const float4* rs = reinterpret_cast<const float4*>(p.R_in + row + c0);
+          if (kMode == kReuse) {
+            const float4* rs = reinterpret_cast<const float4*>(p.R_in + row + c0);
 #pragma unroll
-          for (int c = 0; c < 8; ++c) rr[c] = rs[c];
+            for (int c = 0; c < 8; ++c) rr[c] = rs[c];
+          } else {
+#pragma unroll
+            for (int c = 0; c < 8; ++c) rr[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
           uint4* dst = reinterpret_cast<uint4*>(p.O_out + row + c0);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const float4 r0 = rr[2 * c], r1 = rr[2 * c + 1];
-            const float* v = reinterpret_cast<const float*>(o) + 8 * c;
             uint4 out;
-            out.x = pack_bf16(v[0] * inv + r0.x, v[1] * inv + r0.y);
-            out.y = pack_bf16(v[2] * inv + r0.z, v[3] * inv + r0.w);
-            out.z = pack_bf16(v[4] * inv + r1.x, v[5] * inv + r1.y);
-            out.w = pack_bf16(v[6] * inv + r1.z, v[7] * inv + r1.w);
+            out.x = pack_bf16(__uint_as_float(o[8 * c]) * inv + r0.x,
+                              __uint_as_float(o[8 * c + 1]) * inv + r0.y);
+            out.y = pack_bf16(__uint_as_float(o[8 * c + 2]) * inv + r0.z,
+                              __uint_as_float(o[8 * c + 3]) * inv + r0.w);
+            out.z = pack_bf16(__uint_as_float(o[8 * c + 4]) * inv + r1.x,
+                              __uint_as_float(o[8 * c + 5]) * inv + r1.y);
+            out.w = pack_bf16(__uint_as_float(o[8 * c + 6]) * inv + r1.z,
+                              __uint_as_float(o[8 * c + 7]) * inv + r1.w);
             dst[c] = out;
           }
         }
@@ -464,44 +534,65 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_tc_kernel(const SparsePara
   }
 }
 
-}  // namespace
-
-bool tc_sparse_supported(const AttnArgs& a) { return a.bf16 && a.d == kD; }
-
-template <bool kAnchor>
-static void launch_sparse(const SparseParams& p, int64_t tiles, cudaStream_t st) {
-  cudaFuncSetAttribute(sparse_tc_kernel<kAnchor>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <int kMode>
+void launch(const AttnParams& p, int64_t tiles, cudaStream_t st) {
+  cudaFuncSetAttribute(attn_tc_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)kSmemBytes);
-  sparse_tc_kernel<kAnchor><<<(unsigned)tiles, kThreads, kSmemBytes, st>>>(p);
+  attn_tc_kernel<kMode><<<(unsigned)tiles, kThreads, kSmemBytes, st>>>(p);
 }
 
-int tc_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices,
-              const void* O_full, float* R_out, const float* R_in, void* O_out,
-              cudaStream_t st) {
-  SparseParams p;
+AttnParams base_params(const AttnArgs& a) {
+  AttnParams p{};
   p.Q = (const __nv_bfloat16*)a.Q;
   p.K = (const __nv_bfloat16*)a.K;
   p.V = (const __nv_bfloat16*)a.V;
-  p.groups = groups;
-  p.indices = indices;
   p.n_q = a.n_q;
   p.n_kv = a.n_kv;
   p.gs = a.gs;
   p.G = a.G;
   p.k = a.k;
   p.tiles_per_group = (a.gs + kTile - 1) / kTile;
+  p.q_tiles = (a.n_q + kTile - 1) / kTile;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
+  p.status = a.status;
+  return p;
+}
+
+}  // namespace
+
+bool tc_attention_supported(const AttnArgs& a) { return a.bf16 && a.d == kD; }
+
+int tc_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices,
+              const void* O_full, float* R_out, const float* R_in, void* O_out,
+              cudaStream_t st) {
+  AttnParams p = base_params(a);
+  p.groups = groups;
+  p.indices = indices;
   p.O_full = (const __nv_bfloat16*)O_full;
   p.R_out = R_out;
   p.R_in = R_in;
   p.O_out = (__nv_bfloat16*)O_out;
-  p.status = a.status;
   const int64_t tiles = a.BH * a.G * p.tiles_per_group;
   if (tiles > 0x7fffffffLL) return TLSP_ERR_UNSUPPORTED;
   if (R_out)
-    launch_sparse<true>(p, tiles, st);
+    launch<kAnchor>(p, tiles, st);
   else
-    launch_sparse<false>(p, tiles, st);
+    launch<kReuse>(p, tiles, st);
+  return check_launch();
+}
+
+int tc_dense(const AttnArgs& a, void* O, float* lse, cudaStream_t st) {
+  AttnParams p = base_params(a);
+  if ((uint64_t)a.BH * (uint64_t)std::max(a.n_q, a.n_kv) >= 0x7fffffffull)
+    return TLSP_ERR_UNSUPPORTED;
+  TLSP_TRY(make_tmap_bf16_rows(&p.tmQ, a.Q, (uint64_t)a.BH * a.n_q, kD, 64, kTile));
+  TLSP_TRY(make_tmap_bf16_rows(&p.tmK, a.K, (uint64_t)a.BH * a.n_kv, kD, 64, kTile));
+  TLSP_TRY(make_tmap_bf16_rows(&p.tmV, a.V, (uint64_t)a.BH * a.n_kv, kD, 64, kTile));
+  p.O_out = (__nv_bfloat16*)O;
+  p.lse = lse;
+  const int64_t tiles = a.BH * p.q_tiles;
+  if (tiles > 0x7fffffffLL) return TLSP_ERR_UNSUPPORTED;
+  launch<kDense>(p, tiles, st);
   return check_launch();
 }
 

@@ -45,18 +45,36 @@ int simt_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices
 int make_tmap_bf16_rows(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols,
                         uint32_t box_cols, uint32_t box_rows);
 
-// attn_tc_sparse.cu: tensor-core gathered sparse attention (bf16, d = 128)
-bool tc_sparse_supported(const AttnArgs& a);
+// attn_tc.cu: tensor-core dense pass and gathered sparse pass (bf16, d = 128)
+bool tc_attention_supported(const AttnArgs& a);
 int tc_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices,
               const void* O_full, float* R_out, const float* R_in, void* O_out,
               cudaStream_t st);
+int tc_dense(const AttnArgs& a, void* O, float* lse, cudaStream_t st);
+
+// attn_tc_scores.cu: exact group scores on the tensor cores (bf16, d = 128, g_s <= 128)
+bool tc_scores_supported(const AttnArgs& a);
+int tc_scores(const AttnArgs& a, const int32_t* groups, const float* lse, float* S,
+              cudaStream_t st);
+
+inline int scores_pass(const AttnArgs& a, const int32_t* groups, const float* lse, float* S,
+                       cudaStream_t st) {
+  if (tc_scores_supported(a)) return tc_scores(a, groups, lse, S, st);
+  return simt_scores(a, groups, lse, S, st);
+}
 
 // Sparse pass with the residual epilogue on the best kernel for the shape.
 inline int sparse_pass(const AttnArgs& a, const int32_t* groups, const int32_t* indices,
                        const void* O_full, float* R_out, const float* R_in, void* O_out,
                        cudaStream_t st) {
-  if (tc_sparse_supported(a)) return tc_sparse(a, groups, indices, O_full, R_out, R_in, O_out, st);
+  if (tc_attention_supported(a)) return tc_sparse(a, groups, indices, O_full, R_out, R_in, O_out, st);
   return simt_sparse(a, groups, indices, O_full, R_out, R_in, O_out, st);
+}
+
+// Dense pass (O and the log partition per query) on the best kernel.
+inline int dense_pass(const AttnArgs& a, void* O, float* lse, cudaStream_t st) {
+  if (tc_attention_supported(a)) return tc_dense(a, O, lse, st);
+  return simt_dense(a, O, lse, st);
 }
 
 }  // namespace tlsp

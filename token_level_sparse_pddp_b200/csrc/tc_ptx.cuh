@@ -66,6 +66,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 
 // ------------------------------------------------------------------ TMA
 
+// One box of a 2-D tensor map at (x = column, y = row) into dst; completion
+// counted in bytes on bar. Parts of the box outside the tensor read as zeros.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Four rows r0..r3 x one box of columns starting at col of a 2-D tensor map
 // (box one row high) into four consecutive box rows at dst; completion is
 // counted in bytes on bar. Rows outside the tensor are filled with zeros.
