@@ -147,6 +147,25 @@ int tlsp_anchor_attention(const tlsp_dims* dims, const void* Q, const void* K, c
 int tlsp_dense_attention(const tlsp_dims* dims, const void* Q, const void* K, const void* V,
                          void* O, float* lse, void* ws, size_t ws_bytes, void* stream);
 
+/* Dense attention that allocates nothing (no counterpart in the paper: it is
+ * a convenience of this library). For callers that may not allocate device
+ * memory or pass a workspace, e.g. code running during CUDA graph capture or
+ * under a framework whose pool owns all allocations. Same result as
+ * tlsp_dense_attention with lse = NULL.
+ *   Q, K, V, O   as for tlsp_dense_attention; O is written.
+ * Its scratch (the per-query log partition and a status word) is a fixed
+ * array in the library's device memory, 16 MiB + 256 B, held by every GPU
+ * that loads the library until exit. Limit: B*H*n_q <= 4194304, larger
+ * requests return TLSP_ERR_UNSUPPORTED with nothing launched. The first call
+ * on each device looks the array's address up (with that device current);
+ * make that first call before any stream capture. Every call shares the
+ * array and it keeps the last call's contents: calls that overlap on one GPU
+ * (for instance issued on different streams) race on it. The status word is
+ * cleared at the start of each call; device-side errors recorded there are
+ * not reported. */
+int tlsp_dense_attention_noalloc(const tlsp_dims* dims, const void* Q, const void* K,
+                                 const void* V, void* O, void* stream);
+
 /* Reuse step (review section 3: reuse of the anchor's exact selections and
  * the residual as an additive correction).
  *   Q, K, V   this step's inputs; groups, indices and R from the last anchor.

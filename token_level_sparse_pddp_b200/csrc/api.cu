@@ -52,7 +52,7 @@ static P* at(void* ws, size_t off) {
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
-static int validate_dims(const tlsp_dims* d) {
+int validate_dims(const tlsp_dims* d) {
   if (!d) return TLSP_ERR_INVALID_ARG;
   if (d->batch < 1 || d->heads < 1 || d->n_q < 1 || d->n_kv < 1) return TLSP_ERR_INVALID_ARG;
   if (d->head_dim != 64 && d->head_dim != 128) return TLSP_ERR_INVALID_ARG;

@@ -7,6 +7,9 @@
 
 namespace tlsp {
 
+// ---- api.cu: shape checks shared by the entry points
+int validate_dims(const tlsp_dims* d);
+
 // ---- pddp.cu: tile-aligned query grouping
 struct PddpWork {
   int32_t* perm;      // [BH, n_q] token ids, node segments contiguous

@@ -30,7 +30,8 @@ TLSP_BF16 = 1
 EXPORTED = [
     "tlsp_num_groups", "tlsp_num_levels", "tlsp_workspace_bytes", "tlsp_group_queries",
     "tlsp_group_queries_trace", "tlsp_split_from_projections", "tlsp_anchor_attention",
-    "tlsp_reuse_attention", "tlsp_dense_attention", "tlsp_topk_from_scores", "tlsp_get_device_status",
+    "tlsp_reuse_attention", "tlsp_dense_attention", "tlsp_dense_attention_noalloc",
+    "tlsp_topk_from_scores", "tlsp_get_device_status",
     "tlsp_reset_device_status", "tlsp_debug_bounded_wait", "tlsp_status_string",
     "tlsp_last_cuda_error", "tlsp_launch_count",
 ]
@@ -72,6 +73,7 @@ def lib() -> ctypes.CDLL:
             "tlsp_reuse_attention": (ctypes.c_int,
                                      [dp, vp, vp, vp, vp, i32, i32, vp, vp, vp, vp, sz, vp]),
             "tlsp_dense_attention": (ctypes.c_int, [dp, vp, vp, vp, vp, vp, vp, sz, vp]),
+            "tlsp_dense_attention_noalloc": (ctypes.c_int, [dp, vp, vp, vp, vp, vp]),
             "tlsp_topk_from_scores": (ctypes.c_int, [vp, i32, i32, i32, vp, vp, sz, vp]),
             "tlsp_get_device_status": (ctypes.c_int, [vp]),
             "tlsp_reset_device_status": (ctypes.c_int, [vp, vp]),
@@ -218,6 +220,15 @@ def dense_attention(Q, K, V, ws: Workspace, out=None, lse=None):
     _check(lib().tlsp_dense_attention(ctypes.byref(d), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
                                       _ptr(lse), ws.ptr, ws.nbytes, _stream()),
            "tlsp_dense_attention")
+    return O
+
+
+def dense_attention_noalloc(Q, K, V, out=None):
+    """Dense attention through the entry point that allocates nothing (fixed library scratch)."""
+    d = dims_of(Q, K)
+    O = torch.empty_like(Q) if out is None else out
+    _check(lib().tlsp_dense_attention_noalloc(ctypes.byref(d), _ptr(Q), _ptr(K), _ptr(V), _ptr(O),
+                                              _stream()), "tlsp_dense_attention_noalloc")
     return O
 
 
