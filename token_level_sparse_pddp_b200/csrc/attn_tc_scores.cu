@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) fail(bars, p.status);
       ptx::tc_commit(&bars.drain);
-      ptx::mbar_wait(&bars.drain, 0, abort_flag, kWaitNs);
+      ptx::mbar_wait(&bars.drain, 0, nullptr, kWaitNs);  // even after an abort
     }
     __syncwarp();
   } else if (warp < 4) {
