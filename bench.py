@@ -374,11 +374,12 @@ def main():
 
 
 def tlsp_kernel_rev() -> str:
-    """Hash of the kernel sources: counters taken on other sources are stale."""
+    """Hash of the sources of the sparse attention kernel: counters taken on
+    other sources are stale."""
     import hashlib
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "token_level_sparse_pddp_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in ("attn_tc.cu", "tc_ptx.cuh", "common.cuh", "kernels.h"):
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
 
