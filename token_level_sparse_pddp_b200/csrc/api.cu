@@ -14,7 +14,7 @@ void set_last_cuda_error(cudaError_t e) { t_last_cuda_error = (int)e; }
 
 constexpr size_t kAlign = 256;
 constexpr size_t kStatusBytes = 256;  // status word at 0, debug flag at 64
-constexpr int64_t kPddpPartialSlots = 2048;
+constexpr int64_t kPddpPartialSlots = 640;
 
 static size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -121,7 +121,7 @@ static int group_impl(const tlsp_dims* dims, const void* Q, int32_t gs, int32_t*
   }
   PddpWork w{at<int32_t>(ws, L.perm),    at<int32_t>(ws, L.tmp),   at<uint32_t>(ws, L.seg_key),
              at<float>(ws, L.node_mu),   at<float>(ws, L.node_v),  at<float>(ws, L.partials),
-             kPddpPartialSlots};
+             kPddpPartialSlots,          at<int>(ws, 0)};
   return run_pddp(Q, dims->dtype == TLSP_BF16, dims->head_dim, BH, dims->n_q, gs, groups, proj, w,
                   st);
 }

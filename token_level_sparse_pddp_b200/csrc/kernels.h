@@ -19,6 +19,7 @@ struct PddpWork {
   float* node_v;      // [BH, G, d]
   float* partials;    // [partial_slots, d*d + 2d] chunk moments
   int64_t partial_slots;
+  int* status;        // device status word (timed-out waits)
 };
 int run_pddp(const void* Q, bool bf16, int d, int64_t BH, int n_q, int gs, int32_t* groups,
              float* trace, const PddpWork& w, cudaStream_t st);

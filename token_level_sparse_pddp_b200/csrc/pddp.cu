@@ -8,16 +8,23 @@
 // tokens and `slots` leaf slots sends floor(slots/2)*gs tokens left, so
 // every kernel recomputes a node's (off, cnt, slots) by walking its path bits
 // from the root; no node table is stored. Per level:
-//   1. pddp_moments   (large nodes only) count, mean and centred scatter
+//   1. moments        (large nodes only) count, mean and centred scatter
 //                     matrix of each chunk of a node's rows;
-//   2. pddp_direction combines the chunk moments (pairwise-update formula),
-//                     runs the power iteration and fixes the sign;
-//   3. pddp_project   p_i = (x_i - mu) . v for every token of a split node;
-//   4. pddp_split     radix-select cut at rank floor(slots/2)*gs, stable
+//   2. reduce         combines a node's chunk records (pairwise-update
+//                     formula) into its scatter matrix and mean;
+//   3. direction      power iteration on the scatter matrix (computed in place
+//                     for nodes handled as one chunk), sign fixed;
+//   4. project        p_i = (x_i - mu) . v for every token of a split node;
+//   5. split          radix-select cut at rank floor(slots/2)*gs, stable
 //                     partition of the segment (ties: lower token id).
 // After the last level leaf g is the segment [g*gs, (g+1)*gs) of perm.
+// bf16 inputs with d = 128 take the tensor-core moments and direction kernels;
+// the other shapes take the fp32 SIMT ones. Both write the same records.
+#include <type_traits>
+
 #include "kernels.h"
 #include "select.cuh"
+#include "tc_ptx.cuh"
 
 namespace tlsp {
 
@@ -139,6 +146,47 @@ pddp_moments_kernel(const T* __restrict__ Q, const int32_t* __restrict__ perm, i
   if (threadIdx.x == 0) rec[Moments<D>::kN] = (float)(end - begin);
 }
 
+// Combines the cpn chunk records of a node into record 0 (scatter entries, in
+// place) and node_mu: mu = sum_c n_c mu_c / n and
+// C = sum_c [C_c + n_c (mu_c - mu)(mu_c - mu)^T], both in chunk order. Each CTA
+// owns 256 entries of the D x D scatter; a thread reads and writes only its
+// own entry, so the in-place update has no race.
+template <int D>
+__global__ void __launch_bounds__(256)
+pddp_reduce_kernel(int n_q, int gs, int G, int level, int cpn, float* __restrict__ partials,
+                   float* __restrict__ node_mu) {
+  __shared__ float s_mu[D];
+  const int slice = blockIdx.x, j = blockIdx.y, bh = blockIdx.z, t = threadIdx.x;
+  const NodeDesc nd = node_at(n_q, gs, G, level, j);
+  if (!nd.active) return;
+  float* recs = partials + (int64_t)(bh * (1 << level) + j) * cpn * Moments<D>::kStride;
+  if (t < D) {
+    float s = 0.f, n = 0.f;
+    for (int c = 0; c < cpn; ++c) {
+      const float* rec = recs + (int64_t)c * Moments<D>::kStride;
+      const float nc = rec[Moments<D>::kN];
+      if (nc > 0.f) {
+        s += nc * rec[Moments<D>::kMu + t];
+        n += nc;
+      }
+    }
+    s_mu[t] = s / n;
+  }
+  __syncthreads();
+  const int e = slice * 256 + t, a = e / D, b = e % D;
+  float acc = 0.f;
+  for (int c = 0; c < cpn; ++c) {
+    const float* rec = recs + (int64_t)c * Moments<D>::kStride;
+    const float nc = rec[Moments<D>::kN];
+    if (!(nc > 0.f)) continue;
+    const float da = rec[Moments<D>::kMu + a] - s_mu[a];
+    const float db = rec[Moments<D>::kMu + b] - s_mu[b];
+    acc += rec[e] + nc * da * db;
+  }
+  recs[e] = acc;
+  if (slice == 0 && t < D) node_mu[((int64_t)bh * G + j) * D + t] = s_mu[t];
+}
+
 // Dynamic shared memory of pddp_direction_kernel.
 template <int D>
 constexpr size_t direction_smem_bytes() {
@@ -157,8 +205,7 @@ pddp_direction_kernel(const T* __restrict__ Q, const int32_t* __restrict__ perm,
   float* s_mu = s_rows + kStageRows * D;  // D
   float* s_v = s_mu + D;                  // D
   float* s_w = s_v + D;                   // D
-  float* s_muc = s_w + D;                 // D
-  float* s_red = s_muc + D;               // kMomThreads
+  float* s_red = s_w + D + D;             // kMomThreads
   float* s_misc = s_red + kMomThreads;    // 8
   const int j = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
   const NodeDesc nd = node_at(n_q, gs, G, level, j);
@@ -168,43 +215,13 @@ pddp_direction_kernel(const T* __restrict__ Q, const int32_t* __restrict__ perm,
   if (cpn <= 1) {
     chunk_moments<T, D>(Q + (int64_t)bh * n_q * D, perm + (int64_t)bh * n_q, nd.off,
                         nd.off + nd.cnt, s_rows, s_mu, s_red, acc);
-  } else {
-    const float* recs = partials + (int64_t)(bh * (1 << level) + j) * cpn * Moments<D>::kStride;
-    // overall mean
-    if (t < D) {
-      float s = 0.f, n = 0.f;
-      for (int c = 0; c < cpn; ++c) {
-        const float nc = recs[c * Moments<D>::kStride + Moments<D>::kN];
-        if (nc > 0.f) {
-          s += nc * recs[c * Moments<D>::kStride + Moments<D>::kMu + t];
-          n += nc;
-        }
-      }
-      s_mu[t] = s / n;
-    }
-    __syncthreads();
+  } else {  // scatter and mean combined by pddp_reduce_kernel (record 0, node_mu)
+    const float* rec = partials + (int64_t)(bh * (1 << level) + j) * cpn * Moments<D>::kStride;
+    if (t < D) s_mu[t] = node_mu[((int64_t)bh * G + j) * D + t];
 #pragma unroll
     for (int i = 0; i < BLK; ++i)
 #pragma unroll
-      for (int jj = 0; jj < BLK; ++jj) acc[i][jj] = 0.f;
-    for (int c = 0; c < cpn; ++c) {
-      const float* rec = recs + c * Moments<D>::kStride;
-      const float nc = rec[Moments<D>::kN];
-      if (!(nc > 0.f)) continue;
-      if (t < D) s_muc[t] = rec[Moments<D>::kMu + t] - s_mu[t];
-      __syncthreads();
-      float a[BLK], b[BLK];
-#pragma unroll
-      for (int i = 0; i < BLK; ++i) a[i] = s_muc[bi * BLK + i];
-#pragma unroll
-      for (int jj = 0; jj < BLK; ++jj) b[jj] = s_muc[bj * BLK + jj];
-#pragma unroll
-      for (int i = 0; i < BLK; ++i)
-#pragma unroll
-        for (int jj = 0; jj < BLK; ++jj)
-          acc[i][jj] += rec[(bi * BLK + i) * D + bj * BLK + jj] + nc * a[i] * b[jj];
-      __syncthreads();
-    }
+      for (int jj = 0; jj < BLK; ++jj) acc[i][jj] = rec[(bi * BLK + i) * D + bj * BLK + jj];
   }
 #pragma unroll
   for (int i = 0; i < BLK; ++i)
@@ -252,21 +269,28 @@ pddp_direction_kernel(const T* __restrict__ Q, const int32_t* __restrict__ perm,
   }
 }
 
-// One warp per position of perm: projection of the token there on its node's
-// direction (positions in leaves are skipped).
+// Projection of the token at each position of perm on its node's direction
+// (positions in leaves are skipped). A row is read as 16-byte vectors by a
+// group of D * sizeof(T) / 16 lanes and reduced with shuffles.
 template <class T, int D>
 __global__ void __launch_bounds__(256)
 pddp_project_kernel(const T* __restrict__ Q, const int32_t* __restrict__ perm, int n_q, int gs,
                     int G, int level, const float* __restrict__ node_mu,
                     const float* __restrict__ node_v, uint32_t* __restrict__ seg_key,
                     float* __restrict__ trace, int64_t trace_level_stride) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  constexpr int kVec = 16 / (int)sizeof(T);  // elements per 16-byte load
+  constexpr int kLanes = D / kVec;           // lanes per row (8, 16 or 32)
+  constexpr int kRows = 256 / kLanes;
+  const int sub = threadIdx.x % kLanes;
+  const int pos = blockIdx.x * kRows + threadIdx.x / kLanes;
   const int bh = blockIdx.y;
-  if (warp >= n_q) return;
-  const int pos = warp;
+  bool live = pos < n_q;
   int off = 0, cnt = n_q, slots = G, j = 0;
-  for (int b = 0; b < level; ++b) {
-    if (slots == 1) return;
+  for (int b = 0; b < level && live; ++b) {
+    if (slots == 1) {
+      live = false;
+      break;
+    }
     const int ls = slots / 2, boundary = off + ls * gs;
     if (pos < boundary) {
       cnt = ls * gs;
@@ -279,16 +303,33 @@ pddp_project_kernel(const T* __restrict__ Q, const int32_t* __restrict__ perm, i
       j = 2 * j + 1;
     }
   }
-  if (slots == 1) return;
-  const int token = perm[(int64_t)bh * n_q + pos];
-  const T* x = Q + ((int64_t)bh * n_q + token) * D;
-  const float* mu = node_mu + ((int64_t)bh * G + j) * D;
-  const float* v = node_v + ((int64_t)bh * G + j) * D;
+  live = live && slots > 1;
+  int token = 0;
   float p = 0.f;
+  if (live) {
+    token = perm[(int64_t)bh * n_q + pos];
+    float x[kVec];
+    const T* xp = Q + ((int64_t)bh * n_q + token) * D + sub * kVec;
+    if constexpr (kVec == 8) {
+      load8(xp, x);
+    } else {
+      const float4 u = *reinterpret_cast<const float4*>(xp);
+      x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+    }
+    const float4* mu = reinterpret_cast<const float4*>(node_mu + ((int64_t)bh * G + j) * D + sub * kVec);
+    const float4* v = reinterpret_cast<const float4*>(node_v + ((int64_t)bh * G + j) * D + sub * kVec);
 #pragma unroll
-  for (int c = lane; c < D; c += 32) p = fmaf(to_f32(x[c]) - mu[c], v[c], p);
-  p = warp_sum(p);
-  if (lane == 0) {
+    for (int c = 0; c < kVec / 4; ++c) {
+      const float4 m4 = mu[c], v4 = v[c];
+      p = fmaf(x[4 * c] - m4.x, v4.x, p);
+      p = fmaf(x[4 * c + 1] - m4.y, v4.y, p);
+      p = fmaf(x[4 * c + 2] - m4.z, v4.z, p);
+      p = fmaf(x[4 * c + 3] - m4.w, v4.w, p);
+    }
+  }
+#pragma unroll
+  for (int o = kLanes / 2; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
+  if (live && sub == 0) {
     seg_key[(int64_t)bh * n_q + pos] = float_order_key(p);
     if (trace) trace[level * trace_level_stride + (int64_t)bh * n_q + token] = p;
   }
@@ -316,6 +357,347 @@ pddp_split_kernel(int32_t* __restrict__ perm, int32_t* __restrict__ tmp,
   for (int i = threadIdx.x; i < nd.cnt; i += kSelectThreads) p[i] = o[i];
 }
 
+// ------------------------------------------------------------ tensor-core path
+// bf16 inputs with d = 128. The scatter of a run of rows is the Gram product
+// D^T D of its centred rows d_i = x_i - s, computed on the tensor cores; s is
+// the fp32 mean of the run's first 128 rows, already close to the run's mean.
+// Each d is split into two bf16 parts, d = hi + lo + r with |r| <= 2^-18 |d|,
+// and D^T D ~= hi^T hi + hi^T lo + lo^T hi accumulates in fp32 in TMEM (the
+// dropped lo^T lo term is below 2^-16 of each product). Both operands of each
+// MMA are the same shared-memory tile of 128 rows read MN-major (channels
+// contiguous): A = tile^T (M = channel a, K = row), B = tile (N = channel b).
+// The scatter about the run's own mean is then G - n m m^T, m = mean of d.
+
+constexpr int kGT = 256;  // threads of the tensor-core PDDP kernels
+constexpr int kGD = 128;  // channels
+constexpr int kSub = 128; // rows per MMA batch
+constexpr uint32_t kHalfB = kSub * 128;  // one 64-channel half of a tile: 128 rows x 128 B
+constexpr uint32_t kTileB = 2 * kHalfB;  // one operand (hi or lo), 32 KB
+constexpr uint64_t kGramWaitNs = 1000000000ull;
+
+struct GramShared {
+  float part[16][kGD];  // per row-offset channel sums
+  float shift[kGD];
+  float m[kGD];
+  float v[kGD];
+  float half[2][kGD];
+  float red[8];
+  uint64_t mbar, drain;
+  uint32_t tmem_base;
+};
+constexpr uint32_t kGramSharedB = (sizeof(GramShared) + 1023) / 1024 * 1024;
+constexpr size_t kGramSmem = 1024 + kGramSharedB + 2 * (size_t)kTileB;  // + slack to align
+constexpr size_t kDirSmemNoGram = 1024 + kGramSharedB;
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int k) {
+  return k == 0 ? v.x : k == 1 ? v.y : k == 2 ? v.z : v.w;
+}
+
+// Splits (d0, d1) into packed bf16x2 high parts and low parts.
+__device__ __forceinline__ void split_bf16x2(float d0, float d1, uint32_t& hi, uint32_t& lo) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(d0, d1);
+  hi = *reinterpret_cast<uint32_t*>(&h);
+  __nv_bfloat162 l = __floats2bfloat162_rn(d0 - bf16_lo(hi), d1 - bf16_hi(hi));
+  lo = *reinterpret_cast<uint32_t*>(&l);
+}
+
+// Gram matrix of the rows perm[begin..end) of X ([n_q, 128] bf16, one head)
+// about a shift: TMEM lane a, column b (columns [0,128) at tmem) receives
+// sum_i d_ia d_ib with d_i = x_i - sh.shift. On return sh.m holds the mean of
+// d. Thread t handles the 16-byte chunk t % 16 of rows t / 16 + 16 i; the next
+// batch is loaded into registers while the current one is converted and
+// multiplied. Returns false (status recorded, MMAs drained) after a wait that
+// ran out; the result is the same for every thread of the block.
+__device__ bool gram_tc(const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ perm,
+                        int begin, int end, uint32_t tiles, GramShared& sh, uint32_t tmem,
+                        int* status) {
+  const int t = threadIdx.x;
+  const int q = t & 15, ro = t >> 4;
+  const int h = q >> 3, c8 = q & 7;  // 64-channel half, 16-byte chunk within it
+  const int n = end - begin;
+  const int nsub = (n + kSub - 1) / kSub;
+  const uint4* Xv = reinterpret_cast<const uint4*>(X);
+  uint4 cur[8], nxt[8];
+  auto load = [&](int sub, uint4(&buf)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int r = begin + sub * kSub + ro + 16 * i;
+      buf[i] = r < end ? __ldg(Xv + (int64_t)perm[r] * (kGD / 8) + q) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  load(0, cur);
+  {  // shift: mean of the first batch (rows past the end load as zeros)
+    float s[8] = {};
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        s[2 * k] += bf16_lo(word_of(cur[i], k));
+        s[2 * k + 1] += bf16_hi(word_of(cur[i], k));
+      }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) sh.part[ro][q * 8 + k] = s[k];
+    __syncthreads();
+    if (t < kGD) {
+      float tot = 0.f;
+      for (int r = 0; r < 16; ++r) tot += sh.part[r][t];
+      sh.shift[t] = tot / (float)min(n, kSub);
+    }
+    __syncthreads();
+  }
+  float sv[8], sum[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    sv[k] = sh.shift[q * 8 + k];
+    sum[k] = 0.f;
+  }
+  const uint32_t hi_base = tiles, lo_base = tiles + kTileB;
+  constexpr uint32_t idesc = ptx::idesc_bf16(128, 128, true, true);
+  bool ok = true;
+  for (int sub = 0; sub < nsub; ++sub) {
+    if (sub + 1 < nsub) load(sub + 1, nxt);
+    // the tile is rewritten only after the previous batch's MMAs have read it
+    if (sub > 0) ok = ptx::mbar_wait(&sh.mbar, (sub - 1) & 1, nullptr, kGramWaitNs);
+    if (ok) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = ro + 16 * i;
+        const bool valid = sub * kSub + r < n;
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t x = word_of(cur[i], k);
+          const float d0 = valid ? bf16_lo(x) - sv[2 * k] : 0.f;
+          const float d1 = valid ? bf16_hi(x) - sv[2 * k + 1] : 0.f;
+          sum[2 * k] += d0;
+          sum[2 * k + 1] += d1;
+          split_bf16x2(d0, d1, hw[k], lw[k]);
+        }
+        const uint32_t off = h * kHalfB + r * 128 + ((c8 ^ (r & 7)) << 4);
+        ptx::st_shared_v4(hi_base + off, hw[0], hw[1], hw[2], hw[3]);
+        ptx::st_shared_v4(lo_base + off, lw[0], lw[1], lw[2], lw[3]);
+      }
+    }
+    ptx::fence_proxy_async_smem();
+    ptx::tc_fence_before();
+    if (__syncthreads_or(!ok)) {
+      ok = false;
+      break;
+    }
+    if (t == 0) {
+      ptx::tc_fence_after();
+#pragma unroll
+      for (int ks = 0; ks < kSub / 16; ++ks) {
+        const uint64_t dh = ptx::sw128_desc(hi_base + ks * 2048, kHalfB, 1024);
+        const uint64_t dl = ptx::sw128_desc(lo_base + ks * 2048, kHalfB, 1024);
+        ptx::mma_ss(tmem, dh, dh, idesc, (sub > 0 || ks > 0) ? 1u : 0u);
+        ptx::mma_ss(tmem, dh, dl, idesc, 1u);
+        ptx::mma_ss(tmem, dl, dh, idesc, 1u);
+      }
+      ptx::tc_commit(&sh.mbar);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) cur[i] = nxt[i];
+  }
+  if (ok) ok = ptx::mbar_wait(&sh.mbar, (nsub - 1) & 1, nullptr, kGramWaitNs);
+  if (__syncthreads_or(!ok)) {
+    if (t == 0) {
+      record_status(status, TLSP_ERR_TIMEOUT);
+      ptx::tc_commit(&sh.drain);  // every MMA issued must land before TMEM is freed
+      ptx::mbar_wait(&sh.drain, 0, nullptr, kGramWaitNs);
+    }
+    __syncthreads();
+    return false;
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) sh.part[ro][q * 8 + k] = sum[k];
+  __syncthreads();
+  if (t < kGD) {
+    float tot = 0.f;
+    for (int r = 0; r < 16; ++r) tot += sh.part[r][t];
+    sh.m[t] = tot / (float)n;
+  }
+  __syncthreads();
+  ptx::tc_fence_after();
+  return true;
+}
+
+// Shared-memory carve-up and TMEM allocation common to the two kernels below.
+struct GramCta {
+  GramShared* sh;
+  uint32_t tiles;
+};
+__device__ __forceinline__ GramCta gram_cta_layout(uint8_t* smem_raw) {
+  const uint32_t raw = ptx::smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  return {reinterpret_cast<GramShared*>(smem_raw + (base - raw)), base + kGramSharedB};
+}
+__device__ __forceinline__ uint32_t gram_cta_setup(GramShared& sh) {
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&sh.mbar, 1);
+    ptx::mbar_init(&sh.drain, 1);
+    ptx::fence_mbar_init();
+  }
+  if (threadIdx.x < 32) {
+    ptx::tmem_alloc(&sh.tmem_base, 128);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  return sh.tmem_base;
+}
+__device__ __forceinline__ void gram_cta_release(uint32_t tmem) {
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 128);
+  }
+}
+
+// This thread's 64 entries of the centred scatter held in TMEM: row
+// a = 32 (warp % 4) + lane, columns e0 .. e0 + 63 with e0 = 64 (warp / 4),
+// minus the shift correction n m_a m_b.
+__device__ __forceinline__ void gram_row_part(uint32_t tmem, const GramShared& sh, float n,
+                                              float (&C)[64]) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int a = 32 * (warp & 3) + lane, e0 = 64 * (warp >> 2);
+  const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)e0;
+  uint32_t r0[32], r1[32];
+  ptx::tmem_ld32(tl, r0);
+  ptx::tmem_ld32(tl + 32, r1);
+  ptx::tmem_ld_wait(r0);
+  ptx::reg_barrier(r1);
+  const float nma = n * sh.m[a];
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    C[e] = __uint_as_float(r0[e]) - nma * sh.m[e0 + e];
+    C[32 + e] = __uint_as_float(r1[e]) - nma * sh.m[e0 + 32 + e];
+  }
+}
+
+// Chunk records of the tensor-core path (same format as pddp_moments_kernel).
+__global__ void __launch_bounds__(kGT, 2)
+pddp_gram_tc_kernel(const __nv_bfloat16* __restrict__ Q, const int32_t* __restrict__ perm,
+                    int n_q, int gs, int G, int level, int cpn, float* __restrict__ partials,
+                    int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  const GramCta cta = gram_cta_layout(smem_raw);
+  GramShared& sh = *cta.sh;
+  const int c = blockIdx.x, j = blockIdx.y, bh = blockIdx.z, t = threadIdx.x;
+  const NodeDesc nd = node_at(n_q, gs, G, level, j);
+  if (!nd.active) return;
+  const int len = (nd.cnt + cpn - 1) / cpn;
+  const int begin = nd.off + c * len;
+  const int end = min(nd.off + nd.cnt, begin + len);
+  float* rec = partials + ((int64_t)(bh * (1 << level) + j) * cpn + c) * Moments<kGD>::kStride;
+  if (begin >= end) {
+    if (t == 0) rec[Moments<kGD>::kN] = 0.f;
+    return;
+  }
+  const uint32_t tmem = gram_cta_setup(sh);
+  const bool ok = gram_tc(Q + (int64_t)bh * n_q * kGD, perm + (int64_t)bh * n_q, begin, end,
+                          cta.tiles, sh, tmem, status);
+  if (ok) {
+    float C[64];
+    gram_row_part(tmem, sh, (float)(end - begin), C);
+    const int warp = t >> 5, a = 32 * (warp & 3) + (t & 31), e0 = 64 * (warp >> 2);
+    float4* dst = reinterpret_cast<float4*>(rec + a * kGD + e0);
+#pragma unroll
+    for (int e = 0; e < 64; e += 4) dst[e / 4] = make_float4(C[e], C[e + 1], C[e + 2], C[e + 3]);
+    if (t < kGD) rec[Moments<kGD>::kMu + t] = sh.shift[t] + sh.m[t];
+    if (t == 0) rec[Moments<kGD>::kN] = (float)(end - begin);
+  } else if (t == 0) {
+    rec[Moments<kGD>::kN] = 0.f;
+  }
+  gram_cta_release(tmem);
+}
+
+// Principal direction of one node. With cpn <= 1 the node's scatter is built
+// here (tensor-core Gram over all its rows) and its mean written to node_mu;
+// otherwise both come combined from pddp_reduce_kernel. The scatter stays in
+// registers (thread: row a, 64 columns) for the 16 power iterations
+// v <- C v / |C v|; the sign makes the component of largest magnitude (lowest
+// channel on ties) positive.
+__global__ void __launch_bounds__(kGT, 2)
+pddp_direction_tc_kernel(const __nv_bfloat16* __restrict__ Q, const int32_t* __restrict__ perm,
+                         int n_q, int gs, int G, int level, int cpn,
+                         const float* __restrict__ partials, float* __restrict__ node_mu,
+                         float* __restrict__ node_v, int* status) {
+  extern __shared__ uint8_t smem_raw[];
+  const GramCta cta = gram_cta_layout(smem_raw);
+  GramShared& sh = *cta.sh;
+  const int j = blockIdx.x, bh = blockIdx.y, t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const NodeDesc nd = node_at(n_q, gs, G, level, j);
+  if (!nd.active) return;
+  const int a = 32 * (warp & 3) + lane, e0 = 64 * (warp >> 2);
+  const int64_t node = (int64_t)bh * G + j;
+  float C[64];
+  if (cpn <= 1) {
+    const uint32_t tmem = gram_cta_setup(sh);
+    const bool ok = gram_tc(Q + (int64_t)bh * n_q * kGD, perm + (int64_t)bh * n_q, nd.off,
+                            nd.off + nd.cnt, cta.tiles, sh, tmem, status);
+    if (ok) {
+      gram_row_part(tmem, sh, (float)nd.cnt, C);
+      if (t < kGD) node_mu[node * kGD + t] = sh.shift[t] + sh.m[t];
+    }
+    gram_cta_release(tmem);
+    if (!ok) return;
+  } else {
+    const float4* src = reinterpret_cast<const float4*>(
+        partials + (int64_t)(bh * (1 << level) + j) * cpn * Moments<kGD>::kStride + a * kGD + e0);
+#pragma unroll
+    for (int e = 0; e < 64; e += 4) {
+      const float4 u = src[e / 4];
+      C[e] = u.x;
+      C[e + 1] = u.y;
+      C[e + 2] = u.z;
+      C[e + 3] = u.w;
+    }
+  }
+  if (t < kGD) sh.v[t] = rsqrtf((float)kGD);
+  __syncthreads();
+  for (int it = 0; it < kPowerIters; ++it) {
+    float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;
+#pragma unroll
+    for (int e = 0; e < 64; e += 4) {
+      const float4 vv = *reinterpret_cast<const float4*>(&sh.v[e0 + e]);
+      p0 = fmaf(C[e], vv.x, p0);
+      p1 = fmaf(C[e + 1], vv.y, p1);
+      p2 = fmaf(C[e + 2], vv.z, p2);
+      p3 = fmaf(C[e + 3], vv.w, p3);
+    }
+    sh.half[warp >> 2][a] = (p0 + p1) + (p2 + p3);
+    __syncthreads();
+    float w = 0.f;
+    if (t < kGD) {
+      w = sh.half[0][t] + sh.half[1][t];
+      const float sq = warp_sum(w * w);
+      if (lane == 0) sh.red[warp] = sq;
+    }
+    __syncthreads();
+    const float nw = sqrtf((sh.red[0] + sh.red[1]) + (sh.red[2] + sh.red[3]));
+    if (nw <= 1e-30f * (float)nd.cnt) {  // no spread: e_0 (the same decision in every thread)
+      if (t < kGD) sh.v[t] = t == 0 ? 1.f : 0.f;
+      __syncthreads();
+      break;
+    }
+    if (t < kGD) sh.v[t] = w / nw;
+    __syncthreads();
+  }
+  if (t == 0) {
+    int cmax = 0;
+    for (int c = 1; c < kGD; ++c)
+      if (fabsf(sh.v[c]) > fabsf(sh.v[cmax])) cmax = c;
+    sh.red[4] = sh.v[cmax] < 0.f ? -1.f : 1.f;
+  }
+  __syncthreads();
+  if (t < kGD) node_v[node * kGD + t] = sh.v[t] * sh.red[4];
+}
+
 __global__ void pddp_init_kernel(int32_t* __restrict__ perm, int n_q, int64_t total) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < total) perm[i] = (int32_t)(i % n_q);
@@ -341,32 +723,65 @@ static int levels_of(int G) {
 template <class T, int D>
 static int run_pddp_t(const T* Q, int64_t BH, int n_q, int gs, int32_t* groups, float* trace,
                       const PddpWork& w, cudaStream_t st) {
+  constexpr bool kTc = std::is_same<T, __nv_bfloat16>::value && D == kGD;
   const int G = (n_q + gs - 1) / gs;
   const int L = levels_of(G);
   const int64_t total = BH * n_q;
   pddp_init_kernel<<<(unsigned)ceil_div(total, 256), 256, 0, st>>>(w.perm, n_q, total);
   TLSP_TRY(check_launch());
-  cudaFuncSetAttribute(pddp_direction_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)direction_smem_bytes<D>());
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (kTc) {
+    cudaFuncSetAttribute(pddp_gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)kGramSmem);
+    cudaFuncSetAttribute(pddp_direction_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)kGramSmem);
+  } else {
+    cudaFuncSetAttribute(pddp_direction_kernel<T, D>,
+                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)direction_smem_bytes<D>());
+  }
   for (int level = 0; level < L; ++level) {
-    const int nodes = 1 << level;
+    const int64_t nodes = 1 << level;
     const int64_t max_rows = ceil_div(n_q, nodes) + gs;
-    int64_t cpn = std::min<int64_t>(ceil_div(max_rows, 256), w.partial_slots / (BH * nodes));
+    // Tensor-core path: about two resident CTAs per SM over all chunks, each
+    // chunk at least two MMA batches. SIMT path: chunks of about 256 rows.
+    int64_t cpn = kTc ? std::min<int64_t>(ceil_div(2 * (int64_t)sms, BH * nodes),
+                                          ceil_div(max_rows, 2 * kSub))
+                      : ceil_div(max_rows, 256);
+    cpn = std::min<int64_t>(cpn, w.partial_slots / (BH * nodes));
     if (cpn < 2) cpn = 1;
     if (cpn > 1) {
-      dim3 grid((unsigned)cpn, (unsigned)nodes, (unsigned)BH);
-      pddp_moments_kernel<T, D><<<grid, kMomThreads, 0, st>>>(Q, w.perm, n_q, gs, G, level,
-                                                              (int)cpn, w.partials);
+      const dim3 grid((unsigned)cpn, (unsigned)nodes, (unsigned)BH);
+      if constexpr (kTc) {
+        pddp_gram_tc_kernel<<<grid, kGT, kGramSmem, st>>>(Q, w.perm, n_q, gs, G, level, (int)cpn,
+                                                          w.partials, w.status);
+      } else {
+        pddp_moments_kernel<T, D><<<grid, kMomThreads, 0, st>>>(Q, w.perm, n_q, gs, G, level,
+                                                                (int)cpn, w.partials);
+      }
+      TLSP_TRY(check_launch());
+      pddp_reduce_kernel<D><<<dim3(D * D / 256, (unsigned)nodes, (unsigned)BH), 256, 0, st>>>(
+          n_q, gs, G, level, (int)cpn, w.partials, w.node_mu);
       TLSP_TRY(check_launch());
     }
-    pddp_direction_kernel<T, D><<<dim3(nodes, (unsigned)BH), kMomThreads,
-                                  direction_smem_bytes<D>(), st>>>(
-        Q, w.perm, n_q, gs, G, level, (int)cpn, w.partials, w.node_mu, w.node_v);
+    if constexpr (kTc) {
+      pddp_direction_tc_kernel<<<dim3((unsigned)nodes, (unsigned)BH), kGT,
+                                 cpn > 1 ? kDirSmemNoGram : kGramSmem, st>>>(
+          Q, w.perm, n_q, gs, G, level, (int)cpn, w.partials, w.node_mu, w.node_v, w.status);
+    } else {
+      pddp_direction_kernel<T, D><<<dim3((unsigned)nodes, (unsigned)BH), kMomThreads,
+                                    direction_smem_bytes<D>(), st>>>(
+          Q, w.perm, n_q, gs, G, level, (int)cpn, w.partials, w.node_mu, w.node_v);
+    }
     TLSP_TRY(check_launch());
-    pddp_project_kernel<T, D><<<dim3((unsigned)ceil_div(n_q, 8), (unsigned)BH), 256, 0, st>>>(
-        Q, w.perm, n_q, gs, G, level, w.node_mu, w.node_v, w.seg_key, trace, total);
+    constexpr int kRowsPerBlock = 256 / (D * (int)sizeof(T) / 16);
+    pddp_project_kernel<T, D>
+        <<<dim3((unsigned)ceil_div(n_q, kRowsPerBlock), (unsigned)BH), 256, 0, st>>>(
+            Q, w.perm, n_q, gs, G, level, w.node_mu, w.node_v, w.seg_key, trace, total);
     TLSP_TRY(check_launch());
-    pddp_split_kernel<<<dim3(nodes, (unsigned)BH), kSelectThreads, 0, st>>>(
+    pddp_split_kernel<<<dim3((unsigned)nodes, (unsigned)BH), kSelectThreads, 0, st>>>(
         w.perm, w.tmp, w.seg_key, n_q, gs, G, level);
     TLSP_TRY(check_launch());
   }
