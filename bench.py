@@ -13,9 +13,10 @@ dense-pass times, the reuse-vs-dense speedup, the roofline of the reuse
 kernel, an end-to-end figure through the C ABI with host buffers, and the
 fp64 CPU oracle timed on a bounded sample as a reported baseline.
 
-With --gpus N > 1 (launched by torchrun) every rank runs its own full copy
-of the workload (the path shards by head/batch with no exchange), timings
-are the max over ranks, and `value` aggregates all ranks ("weak" scaling).
+With --gpus N > 1 (launched by torchrun) rank r runs batch elements
+r*B .. r*B + B - 1 of a global batch of N * B (the path shards by batch with
+no exchange), timings are the max over ranks, and `value` aggregates all
+ranks ("weak" scaling).
 `--impl reference` times the oracle on the host cores instead (rank 0 only).
 """
 from __future__ import annotations
@@ -208,31 +209,23 @@ def main():
         return
 
     import torch
-    import torch.distributed as dist
-    from token_level_sparse_pddp_b200 import tlsp
+    from token_level_sparse_pddp_b200 import multi, tlsp
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    info = multi.rank_info()
+    world, rank, local = info.world, info.rank, info.local_rank
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+    multi.init(info, "nccl", device=dev)
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        multi.barrier(info)
 
     def max_over_ranks(vals):
-        t = torch.tensor(vals, dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return t.tolist()
+        return multi.max_over_ranks(info, vals, device=dev)
 
     peaks, peak_kind = load_peaks()
-    it = iter(InputStream(wl, steps=2))
+    # rank r holds batch elements r*B .. r*B + B - 1 of a global batch of world * B
+    it = iter(InputStream(wl, steps=2, batch_offset=multi.batch_offset(wl.batch, rank)))
     _, _, Qa, Ka, Va = next(it)
     _, _, Qr, Kr, Vr = next(it)
     Qa, Ka, Va = (t.to(dev) for t in (Qa, Ka, Va))
@@ -323,7 +316,7 @@ def main():
                          statistics.mean(e2e_ms)])
     total_ms, reuse_mean, anchor_mean, group_mean, dense_mean, e2e_mean = mx
     flops = wl.reuse_flops()
-    value = world * flops / (reuse_mean * 1e-3) / 1e12
+    value = multi.aggregate_rate(flops, world, reuse_mean * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
     achieved = flops / (reuse_mean * 1e-3) / 1e12
     traffic = None
@@ -338,17 +331,18 @@ def main():
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded smooth field + noise)",
-        "config": config_of(wl),
+        "config": dict(config_of(wl), global_batch=world * wl.batch, parallelism=f"dp{world}"),
         "reuse_ms": reuse_mean, "anchor_ms": anchor_mean, "group_queries_ms": group_mean,
         "dense_pass_ms": dense_mean, "reuse_vs_dense_speedup": dense_mean / reuse_mean,
-        "reuse_dense_equiv_tflops": world * wl.dense_flops() / (reuse_mean * 1e-3) / 1e12,
+        "reuse_dense_equiv_tflops": multi.aggregate_rate(wl.dense_flops(), world,
+                                                         reuse_mean * 1e-3) / 1e12,
         "dense_pass_tflops": wl.dense_flops() / (dense_mean * 1e-3) / 1e12,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": "reuse sparse attention (gathered QK^T, PV, +R epilogue)",
                      "peak_kind": f"bf16 dense burst, {peak_kind}",
                      "frac_of_sustained": achieved / float(peaks["bf16_tflops_sustained"])},
-        "e2e": {"value": world * flops / (e2e_mean * 1e-3) / 1e12,
+        "e2e": {"value": multi.aggregate_rate(flops, world, e2e_mean * 1e-3) / 1e12,
                 "unit": "TFLOP/s (executed, reuse step)", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms": e2e_mean},
         "gpu_launches": launches, "clocks": clk,
@@ -369,8 +363,7 @@ def main():
                       f"the GPU's cached k={k} selection + R, fp64) in {el:.1f} s"}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.destroy_process_group()
+    multi.finish(info)
 
 
 def tlsp_kernel_rev() -> str:

@@ -179,7 +179,10 @@ int tlsp_reuse_attention(const tlsp_dims* dims, const void* Q, const void* K, co
 /* Top-k selection on caller-supplied scores (parity hook; the same kernel
  * the anchor step uses).
  *   scores   fp32 [rows, n_kv]; indices out int32 [rows, k], ascending, the k
- *            largest per row with ties to the lower index; -0 equals +0. */
+ *            largest per row with ties to the lower index; -0 equals +0.
+ *   ws       optional (NULL allowed): when given, 16-byte aligned and at least
+ *            256 bytes, a timed-out wait inside the kernel is recorded in its
+ *            status word; ws_bytes is its size. */
 int tlsp_topk_from_scores(const float* scores, int32_t rows, int32_t n_kv, int32_t k,
                           int32_t* indices, void* ws, size_t ws_bytes, void* stream);
 

@@ -191,7 +191,7 @@ int tlsp_anchor_attention(const tlsp_dims* dims, const void* Q, const void* K, c
   float* S = scores ? scores : at<float>(ws, L.scores);
   TLSP_TRY(dense_pass(a, O, lse, st));
   TLSP_TRY(scores_pass(a, groups, lse, S, st));
-  TLSP_TRY(launch_topk(S, a.BH * a.G, a.n_kv, k, indices, st));
+  TLSP_TRY(launch_topk(S, a.BH * a.G, a.n_kv, k, indices, a.status, st));
   return sparse_pass(a, groups, indices, O, R, nullptr, nullptr, st);
 }
 
@@ -224,11 +224,11 @@ int tlsp_reuse_attention(const tlsp_dims* dims, const void* Q, const void* K, co
 
 int tlsp_topk_from_scores(const float* scores, int32_t rows, int32_t n_kv, int32_t k,
                           int32_t* indices, void* ws, size_t ws_bytes, void* stream) {
-  (void)ws;
-  (void)ws_bytes;
   if (!scores || !indices || rows < 0 || n_kv < 1 || k < 1 || k > n_kv)
     return TLSP_ERR_INVALID_ARG;
-  return launch_topk(scores, rows, n_kv, k, indices, (cudaStream_t)stream);
+  if (ws && (!aligned16(ws) || ws_bytes < kStatusBytes)) return TLSP_ERR_INVALID_ARG;
+  int* status = ws ? at<int>(ws, 0) : nullptr;
+  return launch_topk(scores, rows, n_kv, k, indices, status, (cudaStream_t)stream);
 }
 
 int tlsp_get_device_status(const void* ws) {

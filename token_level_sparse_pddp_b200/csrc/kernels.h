@@ -26,7 +26,7 @@ int run_pddp(const void* Q, bool bf16, int d, int64_t BH, int n_q, int gs, int32
 
 // ---- select.cu: top-k and the single PDDP cut
 int launch_topk(const float* scores, int64_t rows, int n_kv, int k, int32_t* indices,
-                cudaStream_t stream);
+                int* status, cudaStream_t stream);
 int launch_split(const float* proj, const int32_t* members, int n, int n_left, int32_t* left,
                  int32_t* right, cudaStream_t stream);
 

@@ -3,13 +3,17 @@
 // MC-Sparse review, section 3: each query group keeps the individual KV
 // tokens of highest exact score, not whole blocks. Ties go to the lower key
 // index and the kept set is listed in ascending key order.
+#include <algorithm>
+
 #include "kernels.h"
 #include "select.cuh"
+#include "tc_ptx.cuh"
 
 namespace tlsp {
 
 // One CTA per score row: the k largest scores (ties: lower index) in
-// ascending key order.
+// ascending key order. Keys are read from global memory on every pass; used
+// when a row does not fit in shared memory.
 __global__ void __launch_bounds__(kSelectThreads)
 topk_rows_kernel(const float* __restrict__ scores, int n_kv, int k, int32_t* __restrict__ indices) {
   __shared__ SelectShared sh;
@@ -20,6 +24,57 @@ topk_rows_kernel(const float* __restrict__ scores, int n_kv, int k, int32_t* __r
   auto key = [&](int i) -> uint32_t { return ~float_order_key(__ldg(s + i)); };
   select_smallest_ordered(
       key, n_kv, k, sh, [&](uint32_t pos, int i) { out[pos] = i; }, [](uint32_t, int) {});
+}
+
+constexpr int kTopkSmemKeys = 46 * 1024;  // rows up to 46K keys are staged (184 KB)
+constexpr uint32_t kBulkChunk = 32768;
+constexpr uint64_t kTopkWaitNs = 1000000000ull;
+
+// Persistent variant: each CTA stages one score row at a time in shared
+// memory (a bulk copy when rows are 16-byte aligned, else plain loads), so
+// every select pass reads shared memory and the row crosses HBM once.
+__global__ void __launch_bounds__(kSelectThreads, 1)
+topk_rows_smem_kernel(const float* __restrict__ scores, int64_t rows, int n_kv, int k,
+                      int32_t* __restrict__ indices, int* status) {
+  extern __shared__ __align__(128) uint8_t topk_smem[];
+  float* buf = reinterpret_cast<float*>(topk_smem);
+  __shared__ SelectShared sh;
+  __shared__ uint64_t bar;
+  const int t = threadIdx.x;
+  const bool bulk = (n_kv % 4) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15u) == 0;
+  if (t == 0) {
+    ptx::mbar_init(&bar, 1);
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  uint32_t phase = 0;
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    const float* s = scores + row * (int64_t)n_kv;
+    if (bulk) {
+      if (t == 0) {
+        const uint32_t bytes = (uint32_t)n_kv * 4u;
+        ptx::fence_proxy_async_smem();
+        ptx::mbar_arrive_expect_tx(&bar, bytes);
+        for (uint32_t off = 0; off < bytes; off += kBulkChunk)
+          ptx::bulk_load(ptx::smem_u32(topk_smem) + off, reinterpret_cast<const uint8_t*>(s) + off,
+                         min(kBulkChunk, bytes - off), &bar);
+      }
+      const bool ok = ptx::mbar_wait(&bar, phase, nullptr, kTopkWaitNs);
+      phase ^= 1u;
+      if (__syncthreads_or(!ok)) {
+        if (t == 0) record_status(status, TLSP_ERR_TIMEOUT);
+        return;
+      }
+    } else {
+      for (int i = t; i < n_kv; i += kSelectThreads) buf[i] = __ldg(s + i);
+      __syncthreads();
+    }
+    int32_t* out = indices + row * (int64_t)k;
+    auto key = [&](int i) -> uint32_t { return ~float_order_key(buf[i]); };
+    select_smallest_ordered(
+        key, n_kv, k, sh, [&](uint32_t pos, int i) { out[pos] = i; }, [](uint32_t, int) {});
+    __syncthreads();  // the row buffer is free for the next row
+  }
 }
 
 // One PDDP cut of `members` (ascending token ids) on projections proj[token].
@@ -34,8 +89,20 @@ split_kernel(const float* __restrict__ proj, const int32_t* __restrict__ members
 }
 
 int launch_topk(const float* scores, int64_t rows, int n_kv, int k, int32_t* indices,
-                cudaStream_t stream) {
+                int* status, cudaStream_t stream) {
   if (rows == 0) return TLSP_OK;
+  if (n_kv <= kTopkSmemKeys) {
+    const size_t smem = (size_t)n_kv * 4;
+    cudaFuncSetAttribute(topk_rows_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)(kTopkSmemKeys * 4));
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t grid = std::min<int64_t>(rows, sms);
+    topk_rows_smem_kernel<<<(unsigned)grid, kSelectThreads, smem, stream>>>(scores, rows, n_kv, k,
+                                                                           indices, status);
+    return check_launch();
+  }
   topk_rows_kernel<<<(unsigned)rows, kSelectThreads, 0, stream>>>(scores, n_kv, k, indices);
   return check_launch();
 }

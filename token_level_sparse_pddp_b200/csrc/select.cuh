@@ -5,8 +5,8 @@
 // ~order(score) over the key index, a PDDP cut on order(projection) over a
 // node whose members are kept in ascending token order. The selection is
 // found by a 3-pass radix select (11 + 11 + 10 bits) on the 32-bit keys and
-// then written out by one in-order pass with block-wide prefix counts, so the
-// selected members come out in position order and the rest in position order.
+// then written out in position order (the selected members, and separately
+// the rest) from per-warp counts over contiguous ranges.
 #pragma once
 
 #include "common.cuh"
@@ -23,26 +23,6 @@ struct SelectShared {
   uint32_t bcast[4];
 };
 
-// Exclusive prefix of a 0/1 flag over the block, plus the block total.
-__device__ __forceinline__ uint32_t block_excl_count(bool flag, uint32_t* warp_tot,
-                                                     uint32_t& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint32_t ballot = __ballot_sync(0xffffffffu, flag);
-  const uint32_t in_warp = __popc(ballot & ((1u << lane) - 1u));
-  if (lane == 0) warp_tot[warp] = __popc(ballot);
-  __syncthreads();
-  uint32_t before = 0, tot = 0;
-#pragma unroll
-  for (int w = 0; w < kSelectThreads / 32; ++w) {
-    const uint32_t c = warp_tot[w];
-    before += (w < warp) ? c : 0u;
-    tot += c;
-  }
-  __syncthreads();
-  total = tot;
-  return before + in_warp;
-}
-
 // Finds the m-th smallest key (1 <= m <= n) among key(0..n-1).
 // On return *T is that key and *need_eq is how many of the keys equal to T
 // (the earliest ones) belong to the m smallest.
@@ -58,9 +38,19 @@ __device__ void radix_select(KeyFn key, int n, int m, SelectShared& sh, uint32_t
     const uint32_t dmask = (1u << widths[pass]) - 1u;
     for (int b = threadIdx.x; b < kRadixBins; b += kSelectThreads) sh.hist[b] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < n; i += kSelectThreads) {
-      const uint32_t k = key(i);
-      if ((k & prefix_mask) == prefix) atomicAdd(&sh.hist[(k >> shift) & dmask], 1u);
+    // Lanes whose keys fall in the same bin add once per warp (match.any):
+    // neighbouring keys often share a bin, and same-address shared atomics
+    // would otherwise serialise.
+    for (int base = 0; base < n; base += kSelectThreads) {
+      const int i = base + threadIdx.x;
+      uint32_t bin = 0xffffffffu;
+      if (i < n) {
+        const uint32_t k = key(i);
+        if ((k & prefix_mask) == prefix) bin = (k >> shift) & dmask;
+      }
+      const uint32_t peers = __match_any_sync(0xffffffffu, bin);
+      if (bin != 0xffffffffu && (int)(threadIdx.x & 31) == __ffs(peers) - 1)
+        atomicAdd(&sh.hist[bin], (uint32_t)__popc(peers));
     }
     __syncthreads();
     // Each thread owns 4 consecutive bins; a block scan of the per-thread sums
@@ -108,39 +98,66 @@ __device__ void radix_select(KeyFn key, int n, int m, SelectShared& sh, uint32_t
 
 // Selects the m smallest of key(0..n-1) (ties to the lower position) and
 // emits them in position order: sel(pos_in_selection, i) for selected i and
-// rest(pos_in_rest, i) for the others. 0 <= m <= n.
+// rest(pos_in_rest, i) for the others. 0 <= m <= n. Each warp owns one
+// contiguous range of positions: a first pass counts its keys below and equal
+// to the threshold, one block-wide exchange turns the counts into starting
+// offsets, and a second pass writes its members with in-warp ballots.
 template <class KeyFn, class SelFn, class RestFn>
 __device__ void select_smallest_ordered(KeyFn key, int n, int m, SelectShared& sh, SelFn sel,
                                         RestFn rest) {
+  constexpr int W = kSelectThreads / 32;
   uint32_t T = 0;
   int need_eq = 0;
-  bool take_all = (m >= n), take_none = (m <= 0);
-  if (!take_all && !take_none) radix_select(key, n, m, sh, &T, &need_eq);
-  uint32_t run_sel = 0, run_eq = 0;
-  for (int base = 0; base < n; base += kSelectThreads) {
-    const int i = base + threadIdx.x;
-    const bool valid = i < n;
-    bool s;
-    if (take_all || take_none) {
-      s = valid && take_all;
-    } else {
-      const uint32_t k = valid ? key(i) : 0xffffffffu;
-      const bool lt = valid && k < T;
-      const bool eq = valid && k == T;
-      uint32_t eq_tot;
-      const uint32_t eq_rank = run_eq + block_excl_count(eq, sh.warp_tot2, eq_tot);
-      run_eq += eq_tot;
-      s = lt || (eq && eq_rank < (uint32_t)need_eq);
+  const bool take_all = (m >= n), take_none = (m <= 0);
+  const bool cut = !take_all && !take_none;
+  if (cut) radix_select(key, n, m, sh, &T, &need_eq);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t below = (1u << lane) - 1u;
+  const int seg = (n + W * 32 - 1) / (W * 32) * 32;
+  const int b0 = min(n, warp * seg), b1 = min(n, b0 + seg);
+  uint32_t sel_run = take_all ? (uint32_t)b0 : 0u, eq_run = 0;
+  if (cut) {
+    uint32_t c_lt = 0, c_eq = 0;
+    for (int base = b0; base < b1; base += 32) {
+      const int i = base + lane;
+      const bool valid = i < b1;
+      const uint32_t k = valid ? key(i) : 0u;
+      c_lt += __popc(__ballot_sync(0xffffffffu, valid && k < T));
+      c_eq += __popc(__ballot_sync(0xffffffffu, valid && k == T));
     }
-    uint32_t sel_tot;
-    const uint32_t pos = run_sel + block_excl_count(s, sh.warp_tot, sel_tot);
+    if (lane == 0) {
+      sh.warp_tot[warp] = c_lt;
+      sh.warp_tot2[warp] = c_eq;
+    }
+    __syncthreads();
+    uint32_t lt_before = 0;
+    for (int w = 0; w < warp; ++w) {
+      lt_before += sh.warp_tot[w];
+      eq_run += sh.warp_tot2[w];
+    }
+    sel_run = lt_before + min(eq_run, (uint32_t)need_eq);
+  }
+  for (int base = b0; base < b1; base += 32) {
+    const int i = base + lane;
+    const bool valid = i < b1;
+    bool s = valid && take_all;
+    if (cut) {
+      const uint32_t k = valid ? key(i) : 0u;
+      const bool eq = valid && k == T;
+      const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
+      const uint32_t eq_rank = eq_run + __popc(eqb & below);
+      eq_run += __popc(eqb);
+      s = (valid && k < T) || (eq && eq_rank < (uint32_t)need_eq);
+    }
+    const uint32_t sb = __ballot_sync(0xffffffffu, s);
+    const uint32_t pos = sel_run + __popc(sb & below);
     if (valid) {
       if (s)
         sel(pos, i);
       else
         rest((uint32_t)i - pos, i);
     }
-    run_sel += sel_tot;
+    sel_run += __popc(sb);
   }
 }
 

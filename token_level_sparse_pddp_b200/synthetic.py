@@ -145,13 +145,18 @@ class InputStream:
     Every (tensor, batch, head) field and every (tensor, batch, head, step)
     drift draws from its own generator spawned from the workload seed, so a
     stream restricted to some heads (`head_ids`) sees exactly the numbers the
-    full stream holds for those heads.
+    full stream holds for those heads. `batch_offset` shifts the batch index
+    the generators are keyed on: a stream with batch_offset = r * B holds
+    batch elements r*B .. r*B + B - 1 of a larger batch (one data-parallel
+    shard of it).
     """
 
-    def __init__(self, wl: Workload, head_ids=None, steps: Optional[int] = None):
+    def __init__(self, wl: Workload, head_ids=None, steps: Optional[int] = None,
+                 batch_offset: int = 0):
         self.wl = wl
         self.head_ids = list(range(wl.heads)) if head_ids is None else list(head_ids)
         self.steps = len(wl.schedule) if steps is None else steps
+        self.batch_offset = int(batch_offset)
 
     def __iter__(self) -> Iterator[Tuple[int, str, torch.Tensor, torch.Tensor, torch.Tensor]]:
         wl = self.wl
@@ -160,20 +165,22 @@ class InputStream:
             range(wl.q_frames[0], wl.q_frames[1] + 1))
         kv_frames = list(range(T))
         nh = len(self.head_ids)
+        b0 = self.batch_offset
         masters = []
         for which, frames in enumerate((q_frames, kv_frames, kv_frames)):
             n = len(frames) * H * W
             m = np.empty((wl.batch, nh, n, wl.head_dim), dtype=np.float32)
             for b in range(wl.batch):
                 for j, h in enumerate(self.head_ids):
-                    m[b, j] = field(_rng(wl.seed, which, b, h), wl.head_dim, wl.grid, frames)
+                    m[b, j] = field(_rng(wl.seed, which, b0 + b, h), wl.head_dim, wl.grid,
+                                    frames)
             masters.append(m)
         for s in range(self.steps):
             if s > 0:
                 for which, m in enumerate(masters):
                     for b in range(wl.batch):
                         for j, h in enumerate(self.head_ids):
-                            g = _rng(wl.seed, which, b, h, s)
+                            g = _rng(wl.seed, which, b0 + b, h, s)
                             m[b, j] += np.float32(wl.drift) * g.standard_normal(
                                 m.shape[2:], dtype=np.float32)
             kind = wl.schedule[s % len(wl.schedule)]

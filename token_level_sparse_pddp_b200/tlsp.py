@@ -232,12 +232,16 @@ def dense_attention_noalloc(Q, K, V, out=None):
     return O
 
 
-def topk_from_scores(scores: torch.Tensor, k: int) -> torch.Tensor:
-    """Per row of fp32 scores [..., n_kv]: ascending indices of the k largest (ties: lower index)."""
+def topk_from_scores(scores: torch.Tensor, k: int, ws: Optional[Workspace] = None) -> torch.Tensor:
+    """Per row of fp32 scores [..., n_kv]: ascending indices of the k largest (ties: lower index).
+
+    With a workspace, a timed-out wait inside the kernel is recorded in its status word."""
     n_kv = scores.shape[-1]
     rows = scores.numel() // n_kv
     idx = torch.empty(scores.shape[:-1] + (k,), dtype=torch.int32, device=scores.device)
-    _check(lib().tlsp_topk_from_scores(_ptr(scores), rows, n_kv, k, _ptr(idx), None, 0, _stream()),
+    wsp, wsn = (ws.ptr, ws.nbytes) if ws is not None else (None, 0)
+    _check(lib().tlsp_topk_from_scores(_ptr(scores), rows, n_kv, k, _ptr(idx), wsp, wsn,
+                                       _stream()),
            "tlsp_topk_from_scores")
     return idx
 
