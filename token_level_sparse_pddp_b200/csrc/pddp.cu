@@ -698,6 +698,34 @@ pddp_direction_tc_kernel(const __nv_bfloat16* __restrict__ Q, const int32_t* __r
   if (t < kGD) node_v[node * kGD + t] = sh.v[t] * sh.red[4];
 }
 
+// pddp_split_kernel with the node's keys staged in shared memory (nodes of
+// at most kSplitSmemKeys tokens). Dynamic shared memory: keys rounded up to 4
+// words, then the radix select's candidate list.
+constexpr int kSplitSmemKeys = 44 * 1024;
+__global__ void __launch_bounds__(kSelectThreads)
+pddp_split_smem_kernel(int32_t* __restrict__ perm, int32_t* __restrict__ tmp,
+                       const uint32_t* __restrict__ seg_key, int n_q, int gs, int G, int level) {
+  extern __shared__ __align__(128) uint8_t split_smem[];
+  __shared__ SelectShared sh;
+  const int j = blockIdx.x, bh = blockIdx.y;
+  const NodeDesc nd = node_at(n_q, gs, G, level, j);
+  if (!nd.active) return;
+  uint32_t* keys = reinterpret_cast<uint32_t*>(split_smem);
+  int* cand = reinterpret_cast<int*>(split_smem + (size_t)((nd.cnt + 3) & ~3) * 4);
+  const int64_t base = (int64_t)bh * n_q + nd.off;
+  for (int i = threadIdx.x; i < nd.cnt; i += kSelectThreads) keys[i] = seg_key[base + i];
+  __syncthreads();
+  const int n_left = (nd.slots / 2) * gs;
+  int32_t* p = perm + base;
+  int32_t* o = tmp + base;
+  smem_select_ordered(
+      keys, nd.cnt, n_left, [](uint32_t w) { return w; }, sh, cand,
+      [&](uint32_t pos, int i) { o[pos] = p[i]; },
+      [&](uint32_t pos, int i) { o[n_left + pos] = p[i]; });
+  __syncthreads();
+  for (int i = threadIdx.x; i < nd.cnt; i += kSelectThreads) p[i] = o[i];
+}
+
 __global__ void pddp_init_kernel(int32_t* __restrict__ perm, int n_q, int64_t total) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < total) perm[i] = (int32_t)(i % n_q);
@@ -737,7 +765,10 @@ static int run_pddp_t(const T* Q, int64_t BH, int n_q, int gs, int32_t* groups, 
                          (int)kGramSmem);
     cudaFuncSetAttribute(pddp_direction_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)kGramSmem);
-  } else {
+  }
+  cudaFuncSetAttribute(pddp_split_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       (int)((size_t)kSplitSmemKeys * 4 + kCandCap * 4));
+  if (!kTc) {
     cudaFuncSetAttribute(pddp_direction_kernel<T, D>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)direction_smem_bytes<D>());
@@ -781,8 +812,14 @@ static int run_pddp_t(const T* Q, int64_t BH, int n_q, int gs, int32_t* groups, 
         <<<dim3((unsigned)ceil_div(n_q, kRowsPerBlock), (unsigned)BH), 256, 0, st>>>(
             Q, w.perm, n_q, gs, G, level, w.node_mu, w.node_v, w.seg_key, trace, total);
     TLSP_TRY(check_launch());
-    pddp_split_kernel<<<dim3((unsigned)nodes, (unsigned)BH), kSelectThreads, 0, st>>>(
-        w.perm, w.tmp, w.seg_key, n_q, gs, G, level);
+    if (max_rows <= kSplitSmemKeys) {
+      const size_t smem = (size_t)((max_rows + 3) & ~3) * 4 + kCandCap * 4;
+      pddp_split_smem_kernel<<<dim3((unsigned)nodes, (unsigned)BH), kSelectThreads, smem, st>>>(
+          w.perm, w.tmp, w.seg_key, n_q, gs, G, level);
+    } else {
+      pddp_split_kernel<<<dim3((unsigned)nodes, (unsigned)BH), kSelectThreads, 0, st>>>(
+          w.perm, w.tmp, w.seg_key, n_q, gs, G, level);
+    }
     TLSP_TRY(check_launch());
   }
   const int64_t out_total = BH * (int64_t)G * gs;

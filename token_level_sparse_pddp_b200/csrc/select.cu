@@ -26,18 +26,26 @@ topk_rows_kernel(const float* __restrict__ scores, int n_kv, int k, int32_t* __r
       key, n_kv, k, sh, [&](uint32_t pos, int i) { out[pos] = i; }, [](uint32_t, int) {});
 }
 
-constexpr int kTopkSmemKeys = 46 * 1024;  // rows up to 46K keys are staged (184 KB)
+constexpr int kTopkSmemKeys = 44 * 1024;  // rows up to 44K keys are staged (176 KB)
 constexpr uint32_t kBulkChunk = 32768;
 constexpr uint64_t kTopkWaitNs = 1000000000ull;
 
+__device__ __forceinline__ uint32_t topk_key(uint32_t w) {
+  // largest score first == smallest complemented order key
+  return ~float_order_key(__uint_as_float(w));
+}
+
 // Persistent variant: each CTA stages one score row at a time in shared
-// memory (a bulk copy when rows are 16-byte aligned, else plain loads), so
-// every select pass reads shared memory and the row crosses HBM once.
+// memory (a bulk copy when rows are 16-byte aligned, else plain loads), so the
+// row crosses HBM once and every pass of the selection reads shared memory.
+// Dynamic shared memory: the row (rounded up to 4 words), then the candidate
+// list of the radix select.
 __global__ void __launch_bounds__(kSelectThreads, 1)
 topk_rows_smem_kernel(const float* __restrict__ scores, int64_t rows, int n_kv, int k,
                       int32_t* __restrict__ indices, int* status) {
   extern __shared__ __align__(128) uint8_t topk_smem[];
-  float* buf = reinterpret_cast<float*>(topk_smem);
+  uint32_t* buf = reinterpret_cast<uint32_t*>(topk_smem);
+  int* cand = reinterpret_cast<int*>(topk_smem + (size_t)((n_kv + 3) & ~3) * 4);
   __shared__ SelectShared sh;
   __shared__ uint64_t bar;
   const int t = threadIdx.x;
@@ -66,16 +74,18 @@ topk_rows_smem_kernel(const float* __restrict__ scores, int64_t rows, int n_kv, 
         return;
       }
     } else {
-      for (int i = t; i < n_kv; i += kSelectThreads) buf[i] = __ldg(s + i);
+      for (int i = t; i < n_kv; i += kSelectThreads) buf[i] = __float_as_uint(__ldg(s + i));
       __syncthreads();
     }
     int32_t* out = indices + row * (int64_t)k;
-    auto key = [&](int i) -> uint32_t { return ~float_order_key(buf[i]); };
-    select_smallest_ordered(
-        key, n_kv, k, sh, [&](uint32_t pos, int i) { out[pos] = i; }, [](uint32_t, int) {});
+    smem_select_ordered(
+        buf, n_kv, k, [](uint32_t w) { return topk_key(w); }, sh, cand,
+        [&](uint32_t pos, int i) { out[pos] = i; }, [](uint32_t, int) {});
     __syncthreads();  // the row buffer is free for the next row
   }
 }
+
+size_t topk_smem_bytes(int n_kv) { return (size_t)((n_kv + 3) & ~3) * 4 + kCandCap * 4; }
 
 // One PDDP cut of `members` (ascending token ids) on projections proj[token].
 __global__ void __launch_bounds__(kSelectThreads)
@@ -92,9 +102,9 @@ int launch_topk(const float* scores, int64_t rows, int n_kv, int k, int32_t* ind
                 int* status, cudaStream_t stream) {
   if (rows == 0) return TLSP_OK;
   if (n_kv <= kTopkSmemKeys) {
-    const size_t smem = (size_t)n_kv * 4;
+    const size_t smem = topk_smem_bytes(n_kv);
     cudaFuncSetAttribute(topk_rows_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)(kTopkSmemKeys * 4));
+                         (int)topk_smem_bytes(kTopkSmemKeys));
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
