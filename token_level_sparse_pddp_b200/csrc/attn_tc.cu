@@ -10,18 +10,22 @@
 //
 // One CTA per 128-query tile: a block of 128 consecutive queries (dense) or
 // a group's queries (sparse; g_s <= 128 is one tile, padding rows are zero and
-// never written back). Warp roles (288 threads, one CTA per SM):
+// never written back). Warp roles (416 threads, one CTA per SM):
 //   warps 0-3  softmax + epilogue: thread t owns query row t = TMEM lane t;
-//   warps 4-7  producers. Dense: lane 0 of warp 4 loads the Q tile and the K
+//   warps 4-11 producers. Dense: lane 0 of warp 4 loads the Q tile and the K
 //              and V tiles of each chunk of 128 keys with TMA box loads.
 //              Sparse: together they load the tile's selection into shared
-//              memory and gather its Q rows, then warps 4-5 gather the K rows
-//              and warps 6-7 the V rows of each chunk of 128 selected keys,
-//              with 16-byte cp.async. Either way the tiles land in 128-byte
-//              swizzled shared memory (the tcgen05 canonical layout);
-//   warp 8     allocates TMEM; lane 0 issues the tcgen05.mma instructions.
+//              memory and gather its Q rows, then warps 4-7 gather the K rows
+//              and warps 8-11 the V rows of each chunk of 128 selected keys,
+//              with 16-byte cp.async (eight issuing warps: the gather rate
+//              grows with the warps that issue, not only with the bytes in
+//              flight). Either way the tiles land in 128-byte swizzled shared
+//              memory (the tcgen05 canonical layout);
+//   warp 12    allocates TMEM; lane 0 issues the tcgen05.mma instructions.
 // Per chunk j: S_j = Q K_j^T (M=N=K=128, fp32 in TMEM), online softmax with
-// exp2 on the SFU, P_j (bf16) written back to TMEM, and O += P_j V_j with A
+// exp2 on the SFU (S read from TMEM 64 columns at a time, the second half
+// loading while the first is processed), P_j (bf16) written back to TMEM,
+// and O += P_j V_j with A
 // read from TMEM and V as an MN-major B operand. TMEM columns: S double
 // buffer [0,256), O [256,384), P double buffer [384,512). K has three
 // shared-memory slots and V two, so loads run ahead of the math.
@@ -44,7 +48,7 @@ enum Mode { kDense = 0, kAnchor = 1, kReuse = 2 };
 
 constexpr int kTile = 128;
 constexpr int kD = 128;
-constexpr int kThreads = 288;
+constexpr int kThreads = 416;
 constexpr uint32_t kTileBytes = kTile * kD * 2;  // 32 KB
 constexpr uint32_t kHalfBytes = kTileBytes / 2;  // one 64-column half: 128 rows x 128 B
 constexpr int kKSlots = 3, kVSlots = 2;
@@ -84,8 +88,45 @@ struct AttnParams {
   const float* __restrict__ R_in;            // reuse
   __nv_bfloat16* __restrict__ O_out;         // dense and reuse
   float* __restrict__ lse;                   // dense: [BH, n_q] natural-log partition
+  int wave;                                  // CTAs resident at once (one per SM)
   int* status;
 };
+
+__device__ __forceinline__ void prefetch_l2(const void* ptr) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+}
+
+// Sparse tiles: pulls into L2 what the prologue and epilogue of tile nb read
+// from HBM: its selection, its query rows and the rows its epilogue reads
+// (R for the reuse step, O_full for the anchor step). Called by the 128
+// producer threads (pt) once their gathers are issued, for the tile one wave
+// ahead, which is the one most likely to start next on some SM; L2 is shared,
+// so it helps wherever that tile runs. Every address lies inside its array.
+template <int kMode>
+__device__ void warm_tile_l2(const AttnParams& p, int64_t nb, int pt) {
+  const int tiles_per_head = p.G * p.tiles_per_group;
+  const int64_t bh = nb / tiles_per_head;
+  const int rem = (int)(nb % tiles_per_head);
+  const int g = rem / p.tiles_per_group, t = rem % p.tiles_per_group;
+  const int32_t* grp = p.groups + (bh * p.G + g) * (int64_t)p.gs;
+  const int32_t* sel = p.indices + (bh * p.G + g) * (int64_t)p.k;
+  for (int q = pt * 32; q < p.k; q += 128 * 32) prefetch_l2(sel + q);
+  if (pt == 0) prefetch_l2(sel + p.k - 1);
+  const int gr = t * kTile + pt;
+  if (gr >= p.gs) return;
+  const int tok = __ldg(grp + gr);
+  if (tok < 0 || tok >= p.n_q) return;
+  const int64_t row = (bh * p.n_q + tok) * kD;
+  prefetch_l2(p.Q + row);
+  prefetch_l2(p.Q + row + 64);
+  if (kMode == kReuse) {
+#pragma unroll
+    for (int l = 0; l < 4; ++l) prefetch_l2(p.R_in + row + 32 * l);
+  } else {
+    prefetch_l2(p.O_full + row);
+    prefetch_l2(p.O_full + row + 64);
+  }
+}
 
 // Row r (0..127) of a [128 x 128] bf16 tile, 16-byte chunk c (0..15), in
 // the 128-byte-swizzled layout: two 64-column halves of 128 rows x 128 B,
@@ -165,13 +206,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_chunks = (n_keys + kTile - 1) / kTile;
 
   if (tid == 0) {
-    ptx::mbar_init(&bars.q_full, kSparse ? 128 : 1);
+    ptx::mbar_init(&bars.q_full, kSparse ? 256 : 1);
     for (int s = 0; s < kKSlots; ++s) {
-      ptx::mbar_init(&bars.k_full[s], kSparse ? 64 : 1);
+      ptx::mbar_init(&bars.k_full[s], kSparse ? 128 : 1);
       ptx::mbar_init(&bars.k_empty[s], 1);
     }
     for (int s = 0; s < kVSlots; ++s) {
-      ptx::mbar_init(&bars.v_full[s], kSparse ? 64 : 1);
+      ptx::mbar_init(&bars.v_full[s], kSparse ? 128 : 1);
       ptx::mbar_init(&bars.v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -184,7 +225,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     bars.abort = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     ptx::tmem_alloc(&bars.tmem_base, kTmCols);
     ptx::tmem_relinquish();
   }
@@ -235,14 +276,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
-  } else if (kSparse && warp >= 4 && warp < 8) {
+  } else if (kSparse && warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ producers
     const int pt = tid - 128;
     // The tile's selection goes to shared memory once (4-byte cp.async by all
     // 128 producers, its own commit group), so no chunk waits on an index load.
     const bool idx_smem = p.k <= kIdxCap;
     if (idx_smem) {
-      for (int q = pt; q < p.k; q += 128)
+      for (int q = pt; q < p.k; q += 256)
         asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(base + kSmIdx + 4u * q),
                      "l"(sel + q)
                      : "memory");
@@ -253,50 +294,52 @@ __global__ void __launch_bounds__(kThreads, 1)
       // all 128 gather Q; then warps 4-5 stream K chunks and warps 6-7 V chunks
       const __nv_bfloat16* Qbh = p.Q + bh * (int64_t)p.n_q * kD;
       {
-        int rows[16];
+        int rows[8];
 #pragma unroll
-        for (int it = 0; it < 16; ++it) {
-          const int gr = t * kTile + it * 8 + (pt >> 4);
+        for (int it = 0; it < 8; ++it) {
+          const int gr = t * kTile + it * 16 + (pt >> 4);
           rows[it] = gr < p.gs ? __ldg(grp + gr) : -1;
         }
 #pragma unroll
-        for (int it = 0; it < 16; ++it) {
+        for (int it = 0; it < 8; ++it) {
           if (rows[it] >= p.n_q) {
             record_status(p.status, TLSP_ERR_DEVICE_ASSERT);
             rows[it] = -1;
           }
         }
-        gather_rows<128>(base + kSmQ, Qbh, rows, pt);
+        gather_rows<256>(base + kSmQ, Qbh, rows, pt);
         ptx::cp_async_arrive_noinc(&bars.q_full);
       }
       if (idx_smem) {
         asm volatile("cp.async.wait_group 0;" ::: "memory");
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        asm volatile("bar.sync 1, 256;" ::: "memory");
       }
       {
-      const bool is_k = warp < 6;
-      const int qt = pt & 63;
+      const bool is_k = warp < 8;
+      const int qt = pt & 127;
       const __nv_bfloat16* src = (is_k ? p.K : p.V) + bh * (int64_t)p.n_kv * kD;
       const int nslots = is_k ? kKSlots : kVSlots;
       const uint32_t slot0 = base + (is_k ? kSmK : kSmV);
       uint64_t* full = is_k ? bars.k_full : bars.v_full;
       uint64_t* empty = is_k ? bars.k_empty : bars.v_empty;
-      int rows[32];
-      chunk_rows<64>(selp, 0, p.k, p.n_kv, qt, rows, p.status);
+      int rows[16];
+      chunk_rows<128>(selp, 0, p.k, p.n_kv, qt, rows, p.status);
       for (int j = 0; j < n_chunks; ++j) {
         const int s = j % nslots, u = j / nslots;
         if (u > 0 && !ptx::mbar_wait(&empty[s], (u - 1) & 1, abort_flag, kWaitNs)) {
           fail(bars, p.status);
           break;
         }
-        gather_rows<64>(slot0 + s * kTileBytes, src, rows, qt);
+        gather_rows<128>(slot0 + s * kTileBytes, src, rows, qt);
         ptx::cp_async_arrive_noinc(&full[s]);
-        if (j + 1 < n_chunks) chunk_rows<64>(selp, j + 1, p.k, p.n_kv, qt, rows, p.status);
+        if (j + 1 < n_chunks) chunk_rows<128>(selp, j + 1, p.k, p.n_kv, qt, rows, p.status);
       }
       }
+      if (pt < 128 && p.wave > 0 && (int64_t)blockIdx.x + p.wave < (int64_t)gridDim.x)
+        warm_tile_l2<kMode>(p, (int64_t)blockIdx.x + p.wave, pt);
       ptx::cp_async_wait_all();
     }
-  } else if (warp == 8) {
+  } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t id_qk = ptx::idesc_bf16(kTile, kTile, false);
@@ -353,6 +396,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int gr = t * kTile + r;
       tok = gr < p.gs ? grp[gr] : -1;
       if (tok >= p.n_q) tok = -1;
+      if (tok >= 0) {  // the row the epilogue reads, towards L2 while the tile computes
+        const int64_t row = (bh * p.n_q + tok) * kD;
+        if (kMode == kReuse) {
+#pragma unroll
+          for (int l = 0; l < 4; ++l) prefetch_l2(p.R_in + row + 32 * l);
+        } else {
+          prefetch_l2(p.O_full + row);
+          prefetch_l2(p.O_full + row + 64);
+        }
+      }
     } else {
       tok = t * kTile + r < p.n_q ? t * kTile + r : -1;
     }
@@ -374,12 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto p_pass = [&](float m_ref, float& sum_out, float& max_out) {
         const float neg_m = -m_ref;
         float sm[4] = {0.f, 0.f, 0.f, 0.f}, mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        uint32_t cur[32], nxt[32];
-        ptx::tmem_ld32(s_col, cur);
-        ptx::tmem_ld_wait(cur);
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          if (b < 3) ptx::tmem_ld32(s_col + 32 * (b + 1), nxt);
+        auto block = [&](const uint32_t (&cur)[32], int b) {
           uint32_t pk[16];
           if (32 * b + 32 <= valid_n) {
 #pragma unroll
@@ -405,12 +453,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           ptx::tmem_st16(p_col + 16 * b, pk);
-          if (b < 3) {
-            ptx::tmem_ld_wait(nxt);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
-          }
-        }
+        };
+        uint32_t ra[32], rb[32];
+        ptx::tmem_ld32(s_col, ra);
+        ptx::tmem_ld32(s_col + 32, rb);
+        ptx::tmem_ld_wait(ra);
+        ptx::reg_barrier(rb);
+        block(ra, 0);
+        ptx::tmem_ld32(s_col + 64, ra);
+        block(rb, 1);
+        ptx::tmem_ld32(s_col + 96, rb);
+        ptx::tmem_ld_wait(ra);
+        ptx::reg_barrier(rb);
+        block(ra, 2);
+        block(rb, 3);
         sum_out = (sm[0] + sm[1]) + (sm[2] + sm[3]);
         max_out = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       };
@@ -463,13 +519,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bars.p_full[s]);
     }
-    // The row this thread finishes is pulled towards L1 while the last PV runs.
     const int64_t row = (bh * p.n_q + (tok >= 0 ? tok : 0)) * kD;
-    if (kMode != kDense && tok >= 0) {
-      const char* pre = kMode == kAnchor ? (const char*)(p.O_full + row) : (const char*)(p.R_in + row);
-      const int lines = kMode == kAnchor ? 2 : 4;
-      for (int l = 0; l < lines; ++l) asm volatile("prefetch.global.L1 [%0];" ::"l"(pre + 128 * l));
-    }
+    // Epilogue operands (R rows for the reuse step, O_full rows for the anchor
+    // step) are read one 32-column block ahead: block 0 before the final wait,
+    // block q + 1 while block q's TMEM load is in flight.
+    const bool has_row = kMode != kDense && tok >= 0;
+    float4 rb[2][8];  // reuse: R, 32 fp32 columns per block
+    uint4 ob[2][4];   // anchor: O_full, 32 bf16 columns per block
+    auto load_block = [&](int q, int b) {
+      if (kMode == kReuse) {
+        const float4* rs = reinterpret_cast<const float4*>(p.R_in + row + q * 32);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) rb[b][c] = rs[c];
+      } else if (kMode == kAnchor) {
+        const uint4* os = reinterpret_cast<const uint4*>(p.O_full + row + q * 32);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ob[b][c] = os[c];
+      }
+    };
+    if (has_row) load_block(0, 0);
     if (ok && !ptx::mbar_wait(&bars.o_final, 0, abort_flag, kWaitNs)) ok = false;
     if (!ok) {
       fail(bars, p.status);
@@ -478,38 +546,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float inv = 1.f / l_run;
       if (kMode == kDense && tok >= 0)  // log partition in natural units: (m + log2 l) ln 2
         p.lse[bh * p.n_q + tok] = (m_run + __log2f(l_run)) * 0.6931471805599453f;
-#pragma unroll 1
+#pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t o[32];
         ptx::tmem_ld32(tl + kTmO + q * 32, o);
+        if (has_row && q < 3) load_block(q + 1, (q + 1) & 1);
         ptx::tmem_ld_wait(o);
         if (tok < 0) continue;
         const int c0 = q * 32;
         if (kMode == kAnchor) {
-          float of[32];
-#pragma unroll
-          for (int c = 0; c < 32; c += 8) load8(p.O_full + row + c0 + c, of + c);
           float4* dst = reinterpret_cast<float4*>(p.R_out + row + c0);
 #pragma unroll
-          for (int c = 0; c < 32; c += 4)
-            dst[c / 4] = make_float4(of[c] - __uint_as_float(o[c]) * inv,
-                                     of[c + 1] - __uint_as_float(o[c + 1]) * inv,
-                                     of[c + 2] - __uint_as_float(o[c + 2]) * inv,
-                                     of[c + 3] - __uint_as_float(o[c + 3]) * inv);
-        } else {
-          float4 rr[8];
-          if (kMode == kReuse) {
-            const float4* rs = reinterpret_cast<const float4*>(p.R_in + row + c0);
+          for (int c = 0; c < 4; ++c) {
+            const uint4 u = ob[q & 1][c];
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-            for (int c = 0; c < 8; ++c) rr[c] = rs[c];
-          } else {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) rr[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int h = 0; h < 2; ++h) {
+              const int e = 8 * c + 4 * h;
+              dst[2 * c + h] = make_float4(
+                  __uint_as_float(w[2 * h] << 16) - __uint_as_float(o[e]) * inv,
+                  __uint_as_float(w[2 * h] & 0xffff0000u) - __uint_as_float(o[e + 1]) * inv,
+                  __uint_as_float(w[2 * h + 1] << 16) - __uint_as_float(o[e + 2]) * inv,
+                  __uint_as_float(w[2 * h + 1] & 0xffff0000u) - __uint_as_float(o[e + 3]) * inv);
+            }
           }
+        } else {
           uint4* dst = reinterpret_cast<uint4*>(p.O_out + row + c0);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            const float4 r0 = rr[2 * c], r1 = rr[2 * c + 1];
+            const float4 r0 = kMode == kReuse ? rb[q & 1][2 * c] : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 r1 =
+                kMode == kReuse ? rb[q & 1][2 * c + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
             uint4 out;
             out.x = pack_bf16(__uint_as_float(o[8 * c]) * inv + r0.x,
                               __uint_as_float(o[8 * c + 1]) * inv + r0.y);
@@ -528,7 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmCols);
   }
@@ -555,6 +622,10 @@ AttnParams base_params(const AttnArgs& a) {
   p.q_tiles = (a.n_q + kTile - 1) / kTile;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
   p.status = a.status;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  p.wave = sms;
   return p;
 }
 

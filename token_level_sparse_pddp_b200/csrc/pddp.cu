@@ -700,8 +700,8 @@ pddp_direction_tc_kernel(const __nv_bfloat16* __restrict__ Q, const int32_t* __r
 
 // pddp_split_kernel with the node's keys staged in shared memory (nodes of
 // at most kSplitSmemKeys tokens). Dynamic shared memory: keys rounded up to 4
-// words, then the radix select's candidate list.
-constexpr int kSplitSmemKeys = 44 * 1024;
+// words.
+constexpr int kSplitSmemKeys = 52 * 1024;
 __global__ void __launch_bounds__(kSelectThreads)
 pddp_split_smem_kernel(int32_t* __restrict__ perm, int32_t* __restrict__ tmp,
                        const uint32_t* __restrict__ seg_key, int n_q, int gs, int G, int level) {
@@ -711,7 +711,6 @@ pddp_split_smem_kernel(int32_t* __restrict__ perm, int32_t* __restrict__ tmp,
   const NodeDesc nd = node_at(n_q, gs, G, level, j);
   if (!nd.active) return;
   uint32_t* keys = reinterpret_cast<uint32_t*>(split_smem);
-  int* cand = reinterpret_cast<int*>(split_smem + (size_t)((nd.cnt + 3) & ~3) * 4);
   const int64_t base = (int64_t)bh * n_q + nd.off;
   for (int i = threadIdx.x; i < nd.cnt; i += kSelectThreads) keys[i] = seg_key[base + i];
   __syncthreads();
@@ -719,7 +718,7 @@ pddp_split_smem_kernel(int32_t* __restrict__ perm, int32_t* __restrict__ tmp,
   int32_t* p = perm + base;
   int32_t* o = tmp + base;
   smem_select_ordered(
-      keys, nd.cnt, n_left, [](uint32_t w) { return w; }, sh, cand,
+      keys, nd.cnt, n_left, [](uint32_t w) { return w; }, sh,
       [&](uint32_t pos, int i) { o[pos] = p[i]; },
       [&](uint32_t pos, int i) { o[n_left + pos] = p[i]; });
   __syncthreads();
@@ -767,7 +766,7 @@ static int run_pddp_t(const T* Q, int64_t BH, int n_q, int gs, int32_t* groups, 
                          (int)kGramSmem);
   }
   cudaFuncSetAttribute(pddp_split_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)((size_t)kSplitSmemKeys * 4 + kCandCap * 4));
+                       (int)((size_t)kSplitSmemKeys * 4));
   if (!kTc) {
     cudaFuncSetAttribute(pddp_direction_kernel<T, D>,
                          cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -813,7 +812,7 @@ static int run_pddp_t(const T* Q, int64_t BH, int n_q, int gs, int32_t* groups, 
             Q, w.perm, n_q, gs, G, level, w.node_mu, w.node_v, w.seg_key, trace, total);
     TLSP_TRY(check_launch());
     if (max_rows <= kSplitSmemKeys) {
-      const size_t smem = (size_t)((max_rows + 3) & ~3) * 4 + kCandCap * 4;
+      const size_t smem = (size_t)((max_rows + 3) & ~3) * 4;
       pddp_split_smem_kernel<<<dim3((unsigned)nodes, (unsigned)BH), kSelectThreads, smem, st>>>(
           w.perm, w.tmp, w.seg_key, n_q, gs, G, level);
     } else {

@@ -26,7 +26,7 @@ topk_rows_kernel(const float* __restrict__ scores, int n_kv, int k, int32_t* __r
       key, n_kv, k, sh, [&](uint32_t pos, int i) { out[pos] = i; }, [](uint32_t, int) {});
 }
 
-constexpr int kTopkSmemKeys = 44 * 1024;  // rows up to 44K keys are staged (176 KB)
+constexpr int kTopkSmemKeys = 52 * 1024;  // rows up to 52K keys are staged (208 KB)
 constexpr uint32_t kBulkChunk = 32768;
 constexpr uint64_t kTopkWaitNs = 1000000000ull;
 
@@ -38,14 +38,12 @@ __device__ __forceinline__ uint32_t topk_key(uint32_t w) {
 // Persistent variant: each CTA stages one score row at a time in shared
 // memory (a bulk copy when rows are 16-byte aligned, else plain loads), so the
 // row crosses HBM once and every pass of the selection reads shared memory.
-// Dynamic shared memory: the row (rounded up to 4 words), then the candidate
-// list of the radix select.
+// Dynamic shared memory: the row, rounded up to 4 words.
 __global__ void __launch_bounds__(kSelectThreads, 1)
 topk_rows_smem_kernel(const float* __restrict__ scores, int64_t rows, int n_kv, int k,
                       int32_t* __restrict__ indices, int* status) {
   extern __shared__ __align__(128) uint8_t topk_smem[];
   uint32_t* buf = reinterpret_cast<uint32_t*>(topk_smem);
-  int* cand = reinterpret_cast<int*>(topk_smem + (size_t)((n_kv + 3) & ~3) * 4);
   __shared__ SelectShared sh;
   __shared__ uint64_t bar;
   const int t = threadIdx.x;
@@ -79,13 +77,13 @@ topk_rows_smem_kernel(const float* __restrict__ scores, int64_t rows, int n_kv, 
     }
     int32_t* out = indices + row * (int64_t)k;
     smem_select_ordered(
-        buf, n_kv, k, [](uint32_t w) { return topk_key(w); }, sh, cand,
+        buf, n_kv, k, [](uint32_t w) { return topk_key(w); }, sh,
         [&](uint32_t pos, int i) { out[pos] = i; }, [](uint32_t, int) {});
     __syncthreads();  // the row buffer is free for the next row
   }
 }
 
-size_t topk_smem_bytes(int n_kv) { return (size_t)((n_kv + 3) & ~3) * 4 + kCandCap * 4; }
+size_t topk_smem_bytes(int n_kv) { return (size_t)((n_kv + 3) & ~3) * 4; }
 
 // One PDDP cut of `members` (ascending token ids) on projections proj[token].
 __global__ void __launch_bounds__(kSelectThreads)

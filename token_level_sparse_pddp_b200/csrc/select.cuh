@@ -158,115 +158,81 @@ __device__ void select_smallest_ordered(KeyFn key, int n, int m, SelectShared& s
 
 // ---------------------------------------------------------------------------
 // The same selection on n words staged in shared memory (16-byte aligned, room
-// for a multiple of 4 words); key_of(word) gives the order key. Every pass
-// reads 16 bytes per lane. Pass 0 builds the histogram of the top 11 bits;
-// pass 1 the next 11 bits of the keys in the chosen bin, and it also lists
-// those keys' positions in `cand` (up to cand_cap), so pass 2 scans only the
-// candidates (all words again if the list overflowed). The output is written
-// by two passes over contiguous per-warp ranges: per-lane counts, then one
-// warp scan per 128 positions.
-
-constexpr int kCandCap = 8192;
+// for a multiple of 4 words). Every pass reads 16 bytes per lane. Pass 0
+// replaces each word by its order key key_of(word) in place and builds the
+// histogram of the top 11 bits; passes 1 and 2 scan the keys again and count
+// only those that share the prefix found so far. The output is written by two
+// passes over contiguous per-warp ranges: per-lane counts, then, per 128
+// positions, four ballots whose popcounts give every member its offset.
 
 template <class KeyOf>
-__device__ void smem_radix_select(const uint32_t* w, int n, int m, KeyOf key_of, SelectShared& sh,
-                                  int* cand, uint32_t* T, int* need_eq) {
-  const int t = threadIdx.x, lane = t & 31;
-  const uint32_t below = (1u << lane) - 1u;
+__device__ void smem_radix_select(uint32_t* w, int n, int m, KeyOf key_of, SelectShared& sh,
+                                  uint32_t* T, int* need_eq) {
+  const int t = threadIdx.x;
   const int n4 = n >> 2;
-  const uint4* w4 = reinterpret_cast<const uint4*>(w);
-  // pass 0: top 11 bits
+  uint4* w4 = reinterpret_cast<uint4*>(w);
   for (int b = t; b < kRadixBins; b += kSelectThreads) sh.hist[b] = 0;
   __syncthreads();
   for (int v = t; v < n4; v += kSelectThreads) {
-    const uint4 u = w4[v];
-    atomicAdd(&sh.hist[key_of(u.x) >> 21], 1u);
-    atomicAdd(&sh.hist[key_of(u.y) >> 21], 1u);
-    atomicAdd(&sh.hist[key_of(u.z) >> 21], 1u);
-    atomicAdd(&sh.hist[key_of(u.w) >> 21], 1u);
+    uint4 u = w4[v];
+    u.x = key_of(u.x);
+    u.y = key_of(u.y);
+    u.z = key_of(u.z);
+    u.w = key_of(u.w);
+    w4[v] = u;
+    atomicAdd(&sh.hist[u.x >> 21], 1u);
+    atomicAdd(&sh.hist[u.y >> 21], 1u);
+    atomicAdd(&sh.hist[u.z >> 21], 1u);
+    atomicAdd(&sh.hist[u.w >> 21], 1u);
   }
-  for (int i = 4 * n4 + t; i < n; i += kSelectThreads) atomicAdd(&sh.hist[key_of(w[i]) >> 21], 1u);
+  for (int i = 4 * n4 + t; i < n; i += kSelectThreads) {
+    w[i] = key_of(w[i]);
+    atomicAdd(&sh.hist[w[i] >> 21], 1u);
+  }
   __syncthreads();
   find_rank_bin(sh, (uint32_t)m);
-  const uint32_t b0 = sh.bcast[0];
+  uint32_t prefix = sh.bcast[0];  // top 11 bits
   uint32_t rank = sh.bcast[1];
   __syncthreads();
-  // pass 1: bits 10..20 of the keys in bin b0, and their positions
-  for (int b = t; b < kRadixBins; b += kSelectThreads) sh.hist[b] = 0;
-  if (t == 0) sh.bcast[2] = 0;
-  __syncthreads();
-  const int n_slots = (n + 3) >> 2;
-  for (int base = 0; base < n_slots; base += kSelectThreads) {
-    const int v = base + t;
-    uint4 u = make_uint4(0, 0, 0, 0);
-    if (v < n_slots) u = w4[v];
-    const uint32_t wq[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int i = 4 * v + q;
-      const uint32_t k = key_of(wq[q]);
-      const bool hit = i < n && (k >> 21) == b0;
-      if (hit) atomicAdd(&sh.hist[(k >> 10) & 0x7ffu], 1u);
-      const uint32_t bal = __ballot_sync(0xffffffffu, hit);
-      if (bal) {
-        uint32_t at = 0;
-        if (lane == __ffs(bal) - 1) at = atomicAdd(&sh.bcast[2], (uint32_t)__popc(bal));
-        at = __shfl_sync(0xffffffffu, at, __ffs(bal) - 1);
-        const uint32_t pos = at + __popc(bal & below);
-        if (hit && pos < (uint32_t)kCandCap) cand[pos] = i;
-      }
+  for (int pass = 1; pass < 3; ++pass) {
+    const int shift = pass == 1 ? 21 : 10;  // keys match when k >> shift == prefix
+    const int dshift = pass == 1 ? 10 : 0;
+    const uint32_t dmask = pass == 1 ? 0x7ffu : 0x3ffu;
+    for (int b = t; b < kRadixBins; b += kSelectThreads) sh.hist[b] = 0;
+    __syncthreads();
+    for (int v = t; v < n4; v += kSelectThreads) {
+      const uint4 u = w4[v];
+      if ((u.x >> shift) == prefix) atomicAdd(&sh.hist[(u.x >> dshift) & dmask], 1u);
+      if ((u.y >> shift) == prefix) atomicAdd(&sh.hist[(u.y >> dshift) & dmask], 1u);
+      if ((u.z >> shift) == prefix) atomicAdd(&sh.hist[(u.z >> dshift) & dmask], 1u);
+      if ((u.w >> shift) == prefix) atomicAdd(&sh.hist[(u.w >> dshift) & dmask], 1u);
     }
+    for (int i = 4 * n4 + t; i < n; i += kSelectThreads)
+      if ((w[i] >> shift) == prefix) atomicAdd(&sh.hist[(w[i] >> dshift) & dmask], 1u);
+    __syncthreads();
+    find_rank_bin(sh, rank);
+    prefix = (prefix << (pass == 1 ? 11 : 10)) | sh.bcast[0];
+    rank = sh.bcast[1];
+    __syncthreads();
   }
-  __syncthreads();
-  const uint32_t n_cand = sh.bcast[2];
-  find_rank_bin(sh, rank);
-  const uint32_t prefix22 = (b0 << 11) | sh.bcast[0];  // top 22 bits
-  rank = sh.bcast[1];
-  __syncthreads();
-  // pass 2: low 10 bits of the keys that share the top 22 bits
-  for (int b = t; b < kRadixBins; b += kSelectThreads) sh.hist[b] = 0;
-  __syncthreads();
-  if (n_cand <= (uint32_t)kCandCap) {
-    for (int c = t; c < (int)n_cand; c += kSelectThreads) {
-      const uint32_t k = key_of(w[cand[c]]);
-      if ((k >> 10) == prefix22) atomicAdd(&sh.hist[k & 0x3ffu], 1u);
-    }
-  } else {
-    for (int i = t; i < n; i += kSelectThreads) {
-      const uint32_t k = key_of(w[i]);
-      if ((k >> 10) == prefix22) atomicAdd(&sh.hist[k & 0x3ffu], 1u);
-    }
-  }
-  __syncthreads();
-  find_rank_bin(sh, rank);
-  *T = (prefix22 << 10) | sh.bcast[0];
-  *need_eq = (int)sh.bcast[1];
-  __syncthreads();
-}
-
-__device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, int lane) {
-  uint32_t incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  return incl - v;
+  *T = prefix;
+  *need_eq = (int)rank;
 }
 
 // Selects the m smallest keys among the n staged words (ties to the lower
 // position), emitting sel(pos_in_selection, i) and rest(pos_in_rest, i) in
-// position order. 0 <= m <= n.
+// position order. 0 <= m <= n. The words are replaced by their keys.
 template <class KeyOf, class SelFn, class RestFn>
-__device__ void smem_select_ordered(const uint32_t* w, int n, int m, KeyOf key_of,
-                                    SelectShared& sh, int* cand, SelFn sel, RestFn rest) {
+__device__ void smem_select_ordered(uint32_t* w, int n, int m, KeyOf key_of, SelectShared& sh,
+                                    SelFn sel, RestFn rest) {
   constexpr int W = kSelectThreads / 32;
   const bool take_all = (m >= n), take_none = (m <= 0);
   const bool cut = !take_all && !take_none;
   uint32_t T = 0;
   int need_eq = 0;
-  if (cut) smem_radix_select(w, n, m, key_of, sh, cand, &T, &need_eq);
+  if (cut) smem_radix_select(w, n, m, key_of, sh, &T, &need_eq);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t below = (1u << lane) - 1u;
   const int n_slots = (n + 3) >> 2;
   const int seg = (n_slots + W - 1) / W;
   const int s0 = min(n_slots, warp * seg), s1 = min(n_slots, s0 + seg);
@@ -276,13 +242,12 @@ __device__ void smem_select_ordered(const uint32_t* w, int n, int m, KeyOf key_o
     uint32_t c_lt = 0, c_eq = 0;
     for (int v = s0 + lane; v < s1; v += 32) {
       const uint4 u = w4[v];
-      const uint32_t wq[4] = {u.x, u.y, u.z, u.w};
+      const uint32_t k4[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const bool valid = 4 * v + q < n;
-        const uint32_t k = key_of(wq[q]);
-        c_lt += (valid && k < T) ? 1u : 0u;
-        c_eq += (valid && k == T) ? 1u : 0u;
+        c_lt += (valid && k4[q] < T) ? 1u : 0u;
+        c_eq += (valid && k4[q] == T) ? 1u : 0u;
       }
     }
     c_lt = __reduce_add_sync(0xffffffffu, c_lt);
@@ -303,40 +268,43 @@ __device__ void smem_select_ordered(const uint32_t* w, int n, int m, KeyOf key_o
     const int v = base + lane;
     uint4 u = make_uint4(0, 0, 0, 0);
     if (v < s1) u = w4[v];
-    const uint32_t wq[4] = {u.x, u.y, u.z, u.w};
+    const uint32_t k4[4] = {u.x, u.y, u.z, u.w};
     bool s[4];
-    uint32_t cs = 0;
     if (cut) {
-      bool lt[4], eq[4];
-      uint32_t ce = 0;
+      bool eq[4];
+      bool any_eq = false;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const bool valid = v < s1 && 4 * v + q < n;
-        const uint32_t k = key_of(wq[q]);
-        lt[q] = valid && k < T;
-        eq[q] = valid && k == T;
-        ce += eq[q] ? 1u : 0u;
+        s[q] = valid && k4[q] < T;
+        eq[q] = valid && k4[q] == T;
+        any_eq |= eq[q];
       }
-      uint32_t eq_rank = eq_run;
-      if (__any_sync(0xffffffffu, ce != 0)) {
-        eq_rank += warp_excl_scan(ce, lane);
-        eq_run += __reduce_add_sync(0xffffffffu, ce);
-      }
+      if (__any_sync(0xffffffffu, any_eq)) {  // ties at the threshold: take the earliest
+        uint32_t eb[4], rank = eq_run;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        s[q] = lt[q] || (eq[q] && eq_rank < (uint32_t)need_eq);
-        eq_rank += eq[q] ? 1u : 0u;
-        cs += s[q] ? 1u : 0u;
+        for (int q = 0; q < 4; ++q) {
+          eb[q] = __ballot_sync(0xffffffffu, eq[q]);
+          rank += __popc(eb[q] & below);
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          s[q] = s[q] || (eq[q] && rank < (uint32_t)need_eq);
+          rank += eq[q] ? 1u : 0u;
+          eq_run += __popc(eb[q]);
+        }
       }
     } else {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        s[q] = take_all && v < s1 && 4 * v + q < n;
-        cs += s[q] ? 1u : 0u;
-      }
+      for (int q = 0; q < 4; ++q) s[q] = take_all && v < s1 && 4 * v + q < n;
     }
-    uint32_t pos = sel_run + warp_excl_scan(cs, lane);
-    sel_run += __reduce_add_sync(0xffffffffu, cs);
+    uint32_t pos = sel_run;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t sb = __ballot_sync(0xffffffffu, s[q]);
+      pos += __popc(sb & below);
+      sel_run += __popc(sb);
+    }
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const int i = 4 * v + q;
