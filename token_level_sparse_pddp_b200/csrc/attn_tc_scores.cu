@@ -14,9 +14,14 @@
 // no cross-thread reduction and no atomics; the per-query LSE (in log2 units)
 // is a shared-memory broadcast. S^T is double-buffered in TMEM so the next
 // chunk's MMA runs while a chunk is summed.
-// Warp roles (288 threads): warps 0-3 sum and store; warps 4-7 gather Q_g
-// with 16-byte cp.async (128-byte swizzle), then lane 0 of warp 4 issues the
-// K loads; warp 8 allocates TMEM and lane 0 issues tcgen05.mma.
+// Warp roles (416 threads): warps 0-3 and 4-7 sum (lane t of both warps w
+// and w + 4 is key j0 + 32 (w % 4) + t; warps 0-3 take the group's query
+// columns 0-63 and warps 4-7 columns 64-127, so two warps per SM sub-partition
+// hide each other's TMEM and SFU latency); warps 4-7 hand their partial sums
+// to warps 0-3 through a double-buffered shared-memory slot, and warps 0-3
+// store the total. Warps 8-11 gather Q_g with 16-byte cp.async (128-byte
+// swizzle), then lane 0 of warp 8 issues the K loads; warp 12 allocates TMEM
+// and lane 0 issues tcgen05.mma.
 // Every wait is bounded (1 s); on expiry the kernel records TLSP_ERR_TIMEOUT
 // and unwinds.
 #include "kernels.h"
@@ -27,14 +32,15 @@ namespace {
 
 constexpr int kTile = 128;
 constexpr int kD = 128;
-constexpr int kThreads = 288;
+constexpr int kThreads = 416;
 constexpr uint32_t kTileBytes = kTile * kD * 2;
 constexpr uint32_t kHalfBytes = kTileBytes / 2;
 constexpr int kKSlots = 4;
 constexpr uint32_t kSmQ = 0, kSmK = kTileBytes;
 constexpr uint32_t kSmBar = (1 + kKSlots) * kTileBytes;
 constexpr uint32_t kSmLse = kSmBar + 256;
-constexpr uint32_t kSmemBytes = kSmLse + kTile * 4 + 1024;
+constexpr uint32_t kSmX = kSmLse + kTile * 4;  // partial sums, 2 x 128 floats
+constexpr uint32_t kSmemBytes = kSmX + 2 * kTile * 4 + 1024;
 constexpr uint32_t kTmCols = 256;
 constexpr uint64_t kWaitNs = 1000000000ull;
 
@@ -42,6 +48,7 @@ struct Bars {
   uint64_t q_full;
   uint64_t k_full[kKSlots], k_empty[kKSlots];
   uint64_t s_full[2], s_empty[2];
+  uint64_t x_full[2], x_empty[2];  // partial sums of warps 4-7 -> warps 0-3
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -93,13 +100,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&bars.s_full[s], 1);
-      ptx::mbar_init(&bars.s_empty[s], 128);
+      ptx::mbar_init(&bars.s_empty[s], 256);
+      ptx::mbar_init(&bars.x_full[s], 128);
+      ptx::mbar_init(&bars.x_empty[s], 128);
     }
     ptx::mbar_init(&bars.drain, 1);
     bars.abort = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     ptx::tmem_alloc(&bars.tmem_base, kTmCols);
     ptx::tmem_relinquish();
   }
@@ -108,9 +117,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
 
-  if (warp >= 4 && warp < 8) {
+  if (warp >= 8 && warp < 12) {
     // ------------------------------------------------------------ producers
-    const int pt = tid - 128;
+    const int pt = tid - 256;
     const __nv_bfloat16* Qbh = p.Q + bh * (int64_t)p.n_q * kD;
     const int c = pt & 15;
 #pragma unroll 1
@@ -134,7 +143,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     ptx::cp_async_arrive_noinc(&bars.q_full);
-    if (warp == 4 && lane == 0) {
+    if (warp == 8 && lane == 0) {
       const int kv_row = (int)(bh * p.n_kv);
       int issued = 0;
       bool ok = true;
@@ -157,7 +166,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     ptx::cp_async_wait_all();
-  } else if (warp == 8) {
+  } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc = ptx::idesc_bf16(kTile, kTile, false);
@@ -185,17 +194,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_wait(&bars.drain, 0, nullptr, kWaitNs);  // even after an abort
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ sums
-    const int r = tid;
-    {
+    const int r = tid & 127, half = warp >> 2;  // key lane r, query columns 64*half ..
+    float* xs = reinterpret_cast<float*>(smem + kSmX);
+    if (half == 0) {
       // log2-unit LSE of the group's queries; padding rows contribute exp2(-inf) = 0
       const int tok = r < p.gs ? grp[r] : -1;
       lse2_s[r] = (tok >= 0 && tok < p.n_q) ? p.lse[bh * p.n_q + tok] * 1.4426950408889634f
                                              : INFINITY;
-      asm volatile("bar.sync 2, 128;" ::: "memory");
     }
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    asm volatile("bar.sync 2, 256;" ::: "memory");
+    float lse2[64];
+#pragma unroll
+    for (int e = 0; e < 64; ++e) lse2[e] = lse2_s[64 * half + e];
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16) + 64 * half;
     float* out = p.S + (bh * p.G + g) * (int64_t)p.n_kv;
     for (int j = 0; j < n_chunks; ++j) {
       const int s = j & 1;
@@ -205,31 +218,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ptx::tc_fence_after();
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t cur[32], nxt[32];
-      ptx::tmem_ld32(tl + s * kTile, cur);
-      ptx::tmem_ld_wait(cur);
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        if (b < 3) ptx::tmem_ld32(tl + s * kTile + 32 * (b + 1), nxt);
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          acc[e & 3] += ptx::ex2(fmaf(__uint_as_float(cur[e]), p.scale_log2, -lse2_s[32 * b + e]));
-        if (b < 3) {
-          ptx::tmem_ld_wait(nxt);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
-        }
-      }
+      uint32_t c0[32], c1[32];
+      ptx::tmem_ld32(tl + s * kTile, c0);
+      ptx::tmem_ld32(tl + s * kTile + 32, c1);
+      ptx::tmem_ld_wait(c0);
+      ptx::reg_barrier(c1);
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars.s_empty[s]);
-      const int key = j * kTile + r;
-      if (key < p.n_kv) out[key] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      ptx::mbar_arrive(&bars.s_empty[s]);  // S is in registers: the MMA may overwrite it
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        acc[e & 3] += ptx::ex2(fmaf(__uint_as_float(c0[e]), p.scale_log2, -lse2[e]));
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        acc[e & 3] += ptx::ex2(fmaf(__uint_as_float(c1[e]), p.scale_log2, -lse2[32 + e]));
+      const float part = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      if (half == 1) {
+        // slot s is free once warps 0-3 have read it for chunk j - 2
+        if (j >= 2 && !ptx::mbar_wait(&bars.x_empty[s], ((j >> 1) - 1) & 1, abort_flag, kWaitNs)) {
+          fail(bars, p.status);
+          break;
+        }
+        xs[s * kTile + r] = part;
+        ptx::mbar_arrive(&bars.x_full[s]);
+      } else {
+        if (!ptx::mbar_wait(&bars.x_full[s], (j >> 1) & 1, abort_flag, kWaitNs)) {
+          fail(bars, p.status);
+          break;
+        }
+        const float total = part + xs[s * kTile + r];
+        ptx::mbar_arrive(&bars.x_empty[s]);
+        const int key = j * kTile + r;
+        if (key < p.n_kv) out[key] = total;
+      }
     }
   }
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, kTmCols);
   }
