@@ -186,6 +186,48 @@ int tlsp_reuse_attention(const tlsp_dims* dims, const void* Q, const void* K, co
 int tlsp_topk_from_scores(const float* scores, int32_t rows, int32_t n_kv, int32_t k,
                           int32_t* indices, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Ablation: the components MC-Sparse replaces (review section 3 and its
+ * ablation table, which adds exact KV selection, token granularity, query
+ * grouping and residual compensation one by one on top of block-sparse
+ * attention with mean-pooled scores). Sparse attention over any selection is
+ * tlsp_reuse_attention (with R = 0 for no residual compensation).
+ * ------------------------------------------------------------------------- */
+
+/* Raster query groups (no PDDP): group g holds tokens g*group_size ..
+ * g*group_size + group_size - 1 in ascending order, -1 past n_q.
+ *   groups  out int32 [B, H, G*group_size]. */
+int tlsp_group_raster(const tlsp_dims* dims, int32_t group_size, int32_t* groups, void* stream);
+
+/* Block-granular selection from per-key scores: keys in blocks of `block`
+ * consecutive tokens; a block's score is the fp32 sum of its keys' scores in
+ * key order; the k / block blocks of largest score (ties to the lower block)
+ * are taken and expanded to their keys, ascending.
+ *   scores        fp32 [rows, n_kv] (for example the exact group scores of
+ *                 the anchor step); indices out int32 [rows, k];
+ *   block_scores  optional out fp32 [rows, n_kv / block] (NULL: not written).
+ * Requires block | n_kv and block | k (else TLSP_ERR_UNSUPPORTED) and
+ * n_kv / block + k / block <= 51200. */
+int tlsp_block_topk_from_scores(const float* scores, int32_t rows, int32_t n_kv, int32_t k,
+                                int32_t block, int32_t* indices, float* block_scores,
+                                void* stream);
+
+/* Block-sparse baseline selection (approximate, mean-pooled scoring): for
+ * each group g and key block m, score = mean(Q rows of g) . mean(K rows of m)
+ * / sqrt(d) in fp32; the k / block best blocks (ties to the lower block) are
+ * expanded to their keys, ascending.
+ *   groups        int32 [B, H, G*group_size] (any grouping, e.g. raster);
+ *   indices       out int32 [B, H, G, k];
+ *   block_scores  optional out fp32 [B, H, G, n_kv / block];
+ *   ws            as for tlsp_anchor_attention (the pooled rows and block
+ *                 scores use its grouping scratch; TLSP_ERR_WORKSPACE if they
+ *                 do not fit).
+ * Requires block | n_kv and block | k (else TLSP_ERR_UNSUPPORTED). */
+int tlsp_pooled_block_select(const tlsp_dims* dims, const void* Q, const void* K,
+                             const int32_t* groups, int32_t group_size, int32_t k, int32_t block,
+                             int32_t* indices, float* block_scores, void* ws, size_t ws_bytes,
+                             void* stream);
+
 /* Device status recorded in `ws` (TLSP_OK, TLSP_ERR_TIMEOUT or
  * TLSP_ERR_DEVICE_ASSERT). Synchronises with the device (blocking copy of the
  * status word): call it after the stream that used `ws` has finished. */

@@ -203,3 +203,49 @@ def reuse_groups(Q, K, V, groups, gs: int, idx_by_group, R_by_group, group_ids=N
         rows = group_rows(groups, gs, g)
         out[g] = sparse(Q[rows], K, V, idx_by_group[g]) + _f64(R_by_group[g])
     return out
+
+
+# ----------------------------------------------------------------- ablation
+# The components MC-Sparse replaces (review section 3 and its ablation table:
+# exact KV selection, token granularity, query grouping and residual
+# compensation added one by one on top of block-sparse attention with
+# mean-pooled scores). Plain numpy, fp64.
+
+def raster_groups(n_q: int, gs: int) -> np.ndarray:
+    """Query groups of consecutive tokens: group g = tokens g*gs .. g*gs + gs - 1, -1 past n_q."""
+    G = -(-n_q // gs)
+    q = np.arange(G * gs)
+    return np.where(q < n_q, q, -1).astype(np.int32)
+
+
+def select_blocks(block_scores, kb: int, b: int) -> np.ndarray:
+    """The kb blocks of largest score (ties to the lower block, ascending), expanded to
+    their b keys each (block m holds keys m*b .. m*b + b - 1), ascending."""
+    blocks = topk(block_scores, kb)
+    return (blocks.astype(np.int64)[:, None] * b + np.arange(b)[None, :]).ravel().astype(np.int32)
+
+
+def block_sums(s, b: int) -> np.ndarray:
+    """Block score of exact per-key scores: the sum over each block of b consecutive keys."""
+    s = _f64(s)
+    return s.reshape(-1, b).sum(axis=1)
+
+
+def block_topk(s, k: int, b: int) -> np.ndarray:
+    """Block-granular exact selection: k / b blocks by summed exact score, expanded."""
+    return select_blocks(block_sums(s, b), k // b, b)
+
+
+def pooled_block_scores(Qg, K, b: int) -> np.ndarray:
+    """Block-sparse baseline scoring: mean of the group's query rows dotted with the
+    mean of each block's key rows, scaled by 1/sqrt(d)."""
+    Qg, K = _f64(Qg), _f64(K)
+    d = K.shape[1]
+    qbar = Qg.mean(axis=0)
+    kbar = K.reshape(-1, b, d).mean(axis=1)
+    return (kbar @ qbar) / np.sqrt(d)
+
+
+def pooled_block_select(Qg, K, k: int, b: int) -> np.ndarray:
+    """Block-sparse baseline selection: k / b blocks by mean-pooled score, expanded."""
+    return select_blocks(pooled_block_scores(Qg, K, b), k // b, b)

@@ -104,4 +104,18 @@ def test_validation_rejects_before_launch(T):
     assert L.tlsp_topk_from_scores(p, 4, 10, 11, p, None, 0, None) == E_ARG
     assert L.tlsp_split_from_projections(p, p, 8, 9, p, p, None, 0, None) == E_ARG
     assert L.tlsp_debug_bounded_wait(None, 0, 10, None) == E_ARG
+    # ablation calls
+    E_UNS = T.TLSP_ERR_UNSUPPORTED
+    assert L.tlsp_group_raster(ctypes.byref(d), 16, None, None) == E_ARG
+    assert L.tlsp_group_raster(ctypes.byref(d), 0, p, None) == E_ARG
+    assert L.tlsp_block_topk_from_scores(p, 4, 128, 129, 4, p, None, None) == E_ARG
+    assert L.tlsp_block_topk_from_scores(p, 4, 128, 32, 0, p, None, None) == E_ARG
+    assert L.tlsp_block_topk_from_scores(p, 4, 128, 32, 5, p, None, None) == E_UNS  # 5 ∤ 128
+    assert L.tlsp_block_topk_from_scores(p, 4, 128, 30, 4, p, None, None) == E_UNS  # 4 ∤ 30
+    assert L.tlsp_pooled_block_select(ctypes.byref(d), p, p, p, 16, 32, 5, p, None, p, big,
+                                      None) == E_UNS
+    assert L.tlsp_pooled_block_select(ctypes.byref(d), p, p, None, 16, 32, 4, p, None, p, big,
+                                      None) == E_ARG
+    assert L.tlsp_pooled_block_select(ctypes.byref(d), p, p, p, 16, 32, 4, p, None, p, 64,
+                                      None) == E_WS
     assert L.tlsp_launch_count() == before

@@ -1,0 +1,116 @@
+"""Ablation of MC-Sparse on the library's own kernels.
+
+    python -m token_level_sparse_pddp_b200.ablation [--workload I] [--block B] [--steps S]
+
+The MC-Sparse review (section 3 and its ablation table) builds the method from
+block-sparse attention with mean-pooled scores by adding, one at a time, exact KV
+selection, token granularity, query grouping and residual compensation. This
+runs that ladder at equal density (k keys per query group) on a workload's
+synthetic schedule and prints, per step and variant, the relative L2 error of the
+output against the library's dense attention (|O - O_dense| / |O_dense| over the
+whole [B, H, n_q, d] tensor) and the device time of the step's selection and
+sparse work:
+
+  bsa           raster query groups, mean-pooled block scores recomputed every
+                step, block-granular selection, no residual;
+  exact_block   raster groups, exact scores on anchor steps (selection cached for
+                the reuse steps), block-granular selection, no residual;
+  exact_token   as exact_block with token-level selection;
+  pddp_token    as exact_token with PDDP query groups;
+  mc_sparse     as pddp_token with the dense-sparse residual R added back.
+
+On an anchor step every variant except bsa runs the dense pass anyway (exact
+scores need it), so its output there is the dense output and the error is 0.
+Every step runs through the C ABI; nothing here computes attention itself.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+from typing import Dict, List
+
+import torch
+
+from . import tlsp
+from .synthetic import InputStream, workload
+
+VARIANTS = ("bsa", "exact_block", "exact_token", "pddp_token", "mc_sparse")
+
+
+def rel_l2(O: torch.Tensor, O_ref: torch.Tensor) -> float:
+    a, r = O.float(), O_ref.float()
+    return float(torch.linalg.vector_norm(a - r) / torch.linalg.vector_norm(r))
+
+
+def run(wl, block: int, steps: int = 0) -> List[Dict]:
+    if wl.n_kv % block or wl.k % block:
+        raise ValueError(f"block {block} must divide n_kv={wl.n_kv} and k={wl.k}")
+    dev = torch.device("cuda")
+    gs, k = wl.group_size, wl.k
+    rows = []
+    ws = None
+    state: Dict[str, Dict] = {v: {} for v in VARIANTS}
+
+    def timed(fn):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        out = fn()
+        b.record()
+        torch.cuda.synchronize()
+        return out, a.elapsed_time(b)
+
+    for s, kind, Q, K, V in InputStream(wl, steps=steps or None):
+        Q, K, V = Q.to(dev), K.to(dev), V.to(dev)
+        if ws is None:
+            ws = tlsp.Workspace(tlsp.dims_of(Q, K), gs, k)
+            raster = tlsp.group_raster(Q, gs)
+            R0 = torch.zeros(Q.shape, dtype=torch.float32, device=dev)
+        O_dense = tlsp.dense_attention(Q, K, V, ws)
+        torch.cuda.synchronize()
+        for v in VARIANTS:
+            st = state[v]
+            if v == "bsa":
+                def step():
+                    idx = tlsp.pooled_block_select(Q, K, raster, gs, k, block, ws)
+                    return tlsp.reuse_attention(Q, K, V, raster, gs, k, idx, R0, ws)
+                O, ms = timed(step)
+            elif kind == "A":
+                def step():
+                    groups = raster if v in ("exact_block", "exact_token") else \
+                        tlsp.group_queries(Q, gs, ws)
+                    O_full, idx, R, S = tlsp.anchor_attention(Q, K, V, groups, gs, k, ws,
+                                                              return_scores=True)
+                    if v == "exact_block":
+                        idx = tlsp.block_topk_from_scores(S, k, block)
+                    return O_full, groups, idx, R
+                (O, groups, idx, R), ms = timed(step)
+                st.update(groups=groups, idx=idx, R=R if v == "mc_sparse" else R0)
+            else:
+                O, ms = timed(lambda: tlsp.reuse_attention(Q, K, V, st["groups"], gs, k,
+                                                           st["idx"], st["R"], ws))
+            if ws.status() != 0:
+                raise RuntimeError(f"device status {tlsp.status_string(ws.status())} in {v}")
+            rows.append(dict(step=s, kind=kind if v != "bsa" else "S", variant=v,
+                             rel_l2=rel_l2(O, O_dense), ms=ms))
+    return rows
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--workload", type=int, default=1)
+    ap.add_argument("--block", type=int, default=0,
+                    help="key block size (default: 64 for workloads 0-1, 104 for 2)")
+    ap.add_argument("--steps", type=int, default=0, help="steps of the schedule (0 = all)")
+    ap.add_argument("--heads", type=int, default=0, help="run with only this many heads")
+    args = ap.parse_args()
+    wl = workload(args.workload)
+    if args.heads:
+        wl = dataclasses.replace(wl, heads=args.heads, name=f"{wl.name}-H{args.heads}")
+    block = args.block or {0: 16, 1: 64, 2: 104}.get(args.workload, 64)
+    for r in run(wl, block, args.steps):
+        print(json.dumps(dict(workload=wl.name, block=block, k=wl.k, **r)), flush=True)
+
+
+if __name__ == "__main__":
+    main()

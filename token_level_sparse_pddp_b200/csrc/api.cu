@@ -231,6 +231,44 @@ int tlsp_topk_from_scores(const float* scores, int32_t rows, int32_t n_kv, int32
   return launch_topk(scores, rows, n_kv, k, indices, status, (cudaStream_t)stream);
 }
 
+int tlsp_group_raster(const tlsp_dims* dims, int32_t group_size, int32_t* groups, void* stream) {
+  TLSP_TRY(validate_dims(dims));
+  TLSP_TRY(validate_grouping(dims, group_size));
+  if (!groups) return TLSP_ERR_INVALID_ARG;
+  return launch_raster_groups(groups, (int64_t)dims->batch * dims->heads, dims->n_q, group_size,
+                              (cudaStream_t)stream);
+}
+
+int tlsp_block_topk_from_scores(const float* scores, int32_t rows, int32_t n_kv, int32_t k,
+                                int32_t block, int32_t* indices, float* block_scores,
+                                void* stream) {
+  if (!scores || !indices || rows < 0 || n_kv < 1 || k < 1 || k > n_kv || block < 1)
+    return TLSP_ERR_INVALID_ARG;
+  if (n_kv % block != 0 || k % block != 0) return TLSP_ERR_UNSUPPORTED;
+  return launch_block_topk(scores, rows, n_kv, n_kv / block, block, k / block, block, indices,
+                           block_scores, (cudaStream_t)stream);
+}
+
+int tlsp_pooled_block_select(const tlsp_dims* dims, const void* Q, const void* K,
+                             const int32_t* groups, int32_t group_size, int32_t k, int32_t block,
+                             int32_t* indices, float* block_scores, void* ws, size_t ws_bytes,
+                             void* stream) {
+  TLSP_TRY(validate_dims(dims));
+  TLSP_TRY(validate_grouping(dims, group_size));
+  if (!Q || !K || !groups || !indices || k < 1 || k > dims->n_kv || block < 1)
+    return TLSP_ERR_INVALID_ARG;
+  if (dims->n_kv % block != 0 || k % block != 0) return TLSP_ERR_UNSUPPORTED;
+  TLSP_TRY(check_ws(dims, group_size, ws, ws_bytes));
+  const Layout L = layout_of(*dims, group_size);
+  const AttnArgs a = attn_args(dims, Q, K, nullptr, group_size, k, ws);
+  // Pooled rows and block scores go to the workspace's chunk-moment region
+  // (grouping scratch, idle during selection).
+  if (pooled_scratch_floats(a, block) * sizeof(float) > L.total - L.partials)
+    return TLSP_ERR_WORKSPACE;
+  return launch_pooled_select(a, groups, block, indices, block_scores, at<float>(ws, L.partials),
+                              (cudaStream_t)stream);
+}
+
 int tlsp_get_device_status(const void* ws) {
   if (!ws) return TLSP_ERR_INVALID_ARG;
   int code = 0;

@@ -30,6 +30,11 @@ int launch_topk(const float* scores, int64_t rows, int n_kv, int k, int32_t* ind
 int launch_split(const float* proj, const int32_t* members, int n, int n_left, int32_t* left,
                  int32_t* right, cudaStream_t stream);
 
+// ---- ablation.cu: the components MC-Sparse replaces
+int launch_raster_groups(int32_t* groups, int64_t BH, int n_q, int gs, cudaStream_t st);
+int launch_block_topk(const float* in, int64_t rows, int n_in, int n_blocks, int sum_width,
+                      int kb, int b_expand, int32_t* indices, float* block_out, cudaStream_t st);
+
 // ---- attention kernels
 struct AttnArgs {
   const void *Q, *K, *V;
@@ -39,6 +44,9 @@ struct AttnArgs {
   int* status;
 };
 int simt_dense(const AttnArgs& a, void* O, float* LSE, cudaStream_t st);
+int launch_pooled_select(const AttnArgs& a, const int32_t* groups, int block, int32_t* indices,
+                         float* block_scores, float* scratch, cudaStream_t st);
+size_t pooled_scratch_floats(const AttnArgs& a, int block);
 int simt_scores(const AttnArgs& a, const int32_t* groups, const float* LSE, float* S,
                 cudaStream_t st);
 int simt_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices,

@@ -33,7 +33,8 @@ EXPORTED = [
     "tlsp_reuse_attention", "tlsp_dense_attention", "tlsp_dense_attention_noalloc",
     "tlsp_topk_from_scores", "tlsp_get_device_status",
     "tlsp_reset_device_status", "tlsp_debug_bounded_wait", "tlsp_status_string",
-    "tlsp_last_cuda_error", "tlsp_launch_count",
+    "tlsp_last_cuda_error", "tlsp_launch_count", "tlsp_group_raster",
+    "tlsp_block_topk_from_scores", "tlsp_pooled_block_select",
 ]
 
 
@@ -81,6 +82,10 @@ def lib() -> ctypes.CDLL:
             "tlsp_status_string": (ctypes.c_char_p, [ctypes.c_int]),
             "tlsp_last_cuda_error": (ctypes.c_int, []),
             "tlsp_launch_count": (i64, []),
+            "tlsp_group_raster": (ctypes.c_int, [dp, i32, vp, vp]),
+            "tlsp_block_topk_from_scores": (ctypes.c_int, [vp, i32, i32, i32, i32, vp, vp, vp]),
+            "tlsp_pooled_block_select": (ctypes.c_int,
+                                         [dp, vp, vp, vp, i32, i32, i32, vp, vp, vp, sz, vp]),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -261,3 +266,46 @@ def split_from_projections(proj: torch.Tensor, members: torch.Tensor,
 def debug_bounded_wait(ws: Workspace, spin_limit: int):
     _check(lib().tlsp_debug_bounded_wait(ws.ptr, ws.nbytes, spin_limit, _stream()),
            "tlsp_debug_bounded_wait")
+
+
+# ----------------------------------------------------------------- ablation
+
+def group_raster(Q: torch.Tensor, group_size: int, out: Optional[torch.Tensor] = None):
+    """Raster query groups (consecutive tokens, no PDDP) -> int32 [B, H, G*group_size]."""
+    d = dims_of(Q)
+    G = num_groups(d.n_q, group_size)
+    groups = (torch.empty((d.batch, d.heads, G * group_size), dtype=torch.int32, device=Q.device)
+              if out is None else out)
+    _check(lib().tlsp_group_raster(ctypes.byref(d), group_size, _ptr(groups), _stream()),
+           "tlsp_group_raster")
+    return groups
+
+
+def block_topk_from_scores(scores: torch.Tensor, k: int, block: int,
+                           return_block_scores: bool = False):
+    """Block-granular selection from per-key scores [..., n_kv] -> indices [..., k]
+    (and the block scores [..., n_kv / block] when asked)."""
+    n_kv = scores.shape[-1]
+    rows = scores.numel() // n_kv
+    idx = torch.empty(scores.shape[:-1] + (k,), dtype=torch.int32, device=scores.device)
+    bs = (torch.empty(scores.shape[:-1] + (n_kv // block,), dtype=torch.float32,
+                      device=scores.device) if return_block_scores else None)
+    _check(lib().tlsp_block_topk_from_scores(_ptr(scores), rows, n_kv, k, block, _ptr(idx),
+                                             _ptr(bs), _stream()),
+           "tlsp_block_topk_from_scores")
+    return (idx, bs) if return_block_scores else idx
+
+
+def pooled_block_select(Q: torch.Tensor, K: torch.Tensor, groups: torch.Tensor, group_size: int,
+                        k: int, block: int, ws: Workspace, return_block_scores: bool = False):
+    """Block-sparse baseline selection (mean-pooled block scores) -> indices [B, H, G, k]."""
+    d = dims_of(Q, K)
+    G = num_groups(d.n_q, group_size)
+    idx = torch.empty((d.batch, d.heads, G, k), dtype=torch.int32, device=Q.device)
+    bs = (torch.empty((d.batch, d.heads, G, d.n_kv // block), dtype=torch.float32,
+                      device=Q.device) if return_block_scores else None)
+    _check(lib().tlsp_pooled_block_select(ctypes.byref(d), _ptr(Q), _ptr(K), _ptr(groups),
+                                          group_size, k, block, _ptr(idx), _ptr(bs), ws.ptr,
+                                          ws.nbytes, _stream()),
+           "tlsp_pooled_block_select")
+    return (idx, bs) if return_block_scores else idx
