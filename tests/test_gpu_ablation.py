@@ -150,3 +150,14 @@ def test_ablation_all_keys_is_dense(T):
     wl = Workload("abl-all", 1, 2, 128, (2, 8, 8), None, "bf16", 16, 128, "ARR", 0.05, 13)
     for r in ablation.run(wl, 32):
         assert r["rel_l2"] <= 5e-3, r
+
+
+def test_error_decomposition_structure(T):
+    """Each rung adds an error source; with every key selected all rungs are dense."""
+    from token_level_sparse_pddp_b200 import ablation
+    rows = ablation.decompose(workload(1), 64)
+    assert [r["component"] for r in rows] == [c for c, _ in ablation.DECOMPOSITION]
+    assert all(np.isfinite(r["rel_l2"]) and r["rel_l2"] > 0 for r in rows)
+    wl = Workload("dec-all", 1, 2, 128, (2, 8, 8), None, "bf16", 16, 128, "A", 0.0, 17)
+    for r in ablation.decompose(wl, 32):
+        assert r["rel_l2"] <= 5e-3, r
