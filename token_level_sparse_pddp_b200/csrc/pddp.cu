@@ -271,7 +271,11 @@ pddp_direction_kernel(const T* __restrict__ Q, const int32_t* __restrict__ perm,
 
 // Projection of the token at each position of perm on its node's direction
 // (positions in leaves are skipped). A row is read as 16-byte vectors by a
-// group of D * sizeof(T) / 16 lanes and reduced with shuffles.
+// group of D * sizeof(T) / 16 lanes and reduced with shuffles; each group
+// takes kProjRows rows and issues all their loads before it uses any, so the
+// perm -> row -> reduce chains of the rows overlap.
+constexpr int kProjRows = 4;
+
 template <class T, int D>
 __global__ void __launch_bounds__(256)
 pddp_project_kernel(const T* __restrict__ Q, const int32_t* __restrict__ perm, int n_q, int gs,
@@ -280,58 +284,71 @@ pddp_project_kernel(const T* __restrict__ Q, const int32_t* __restrict__ perm, i
                     float* __restrict__ trace, int64_t trace_level_stride) {
   constexpr int kVec = 16 / (int)sizeof(T);  // elements per 16-byte load
   constexpr int kLanes = D / kVec;           // lanes per row (8, 16 or 32)
-  constexpr int kRows = 256 / kLanes;
+  constexpr int kRows = 256 / kLanes;        // rows per pass of the block
   const int sub = threadIdx.x % kLanes;
-  const int pos = blockIdx.x * kRows + threadIdx.x / kLanes;
   const int bh = blockIdx.y;
-  bool live = pos < n_q;
-  int off = 0, cnt = n_q, slots = G, j = 0;
-  for (int b = 0; b < level && live; ++b) {
-    if (slots == 1) {
-      live = false;
-      break;
+  int pos[kProjRows], node[kProjRows], token[kProjRows];
+  bool live[kProjRows];
+#pragma unroll
+  for (int q = 0; q < kProjRows; ++q) {
+    pos[q] = (blockIdx.x * kProjRows + q) * kRows + threadIdx.x / kLanes;
+    live[q] = pos[q] < n_q;
+    int off = 0, slots = G, j = 0;
+    for (int b = 0; b < level && live[q]; ++b) {
+      if (slots == 1) break;
+      const int ls = slots / 2, boundary = off + ls * gs;
+      if (pos[q] < boundary) {
+        slots = ls;
+        j = 2 * j;
+      } else {
+        off = boundary;
+        slots -= ls;
+        j = 2 * j + 1;
+      }
     }
-    const int ls = slots / 2, boundary = off + ls * gs;
-    if (pos < boundary) {
-      cnt = ls * gs;
-      slots = ls;
-      j = 2 * j;
-    } else {
-      off = boundary;
-      cnt -= ls * gs;
-      slots -= ls;
-      j = 2 * j + 1;
-    }
+    live[q] = live[q] && slots > 1;
+    node[q] = j;
+    token[q] = live[q] ? perm[(int64_t)bh * n_q + pos[q]] : 0;
   }
-  live = live && slots > 1;
-  int token = 0;
-  float p = 0.f;
-  if (live) {
-    token = perm[(int64_t)bh * n_q + pos];
-    float x[kVec];
-    const T* xp = Q + ((int64_t)bh * n_q + token) * D + sub * kVec;
+  float x[kProjRows][kVec];
+#pragma unroll
+  for (int q = 0; q < kProjRows; ++q) {
+    const T* xp = Q + ((int64_t)bh * n_q + token[q]) * D + sub * kVec;
     if constexpr (kVec == 8) {
-      load8(xp, x);
+      load8(xp, x[q]);
     } else {
       const float4 u = *reinterpret_cast<const float4*>(xp);
-      x[0] = u.x; x[1] = u.y; x[2] = u.z; x[3] = u.w;
+      x[q][0] = u.x; x[q][1] = u.y; x[q][2] = u.z; x[q][3] = u.w;
     }
-    const float4* mu = reinterpret_cast<const float4*>(node_mu + ((int64_t)bh * G + j) * D + sub * kVec);
-    const float4* v = reinterpret_cast<const float4*>(node_v + ((int64_t)bh * G + j) * D + sub * kVec);
+  }
+  float p[kProjRows];
+#pragma unroll
+  for (int q = 0; q < kProjRows; ++q) {
+    p[q] = 0.f;
+    const float4* mu =
+        reinterpret_cast<const float4*>(node_mu + ((int64_t)bh * G + node[q]) * D + sub * kVec);
+    const float4* v =
+        reinterpret_cast<const float4*>(node_v + ((int64_t)bh * G + node[q]) * D + sub * kVec);
 #pragma unroll
     for (int c = 0; c < kVec / 4; ++c) {
       const float4 m4 = mu[c], v4 = v[c];
-      p = fmaf(x[4 * c] - m4.x, v4.x, p);
-      p = fmaf(x[4 * c + 1] - m4.y, v4.y, p);
-      p = fmaf(x[4 * c + 2] - m4.z, v4.z, p);
-      p = fmaf(x[4 * c + 3] - m4.w, v4.w, p);
+      p[q] = fmaf(x[q][4 * c] - m4.x, v4.x, p[q]);
+      p[q] = fmaf(x[q][4 * c + 1] - m4.y, v4.y, p[q]);
+      p[q] = fmaf(x[q][4 * c + 2] - m4.z, v4.z, p[q]);
+      p[q] = fmaf(x[q][4 * c + 3] - m4.w, v4.w, p[q]);
     }
   }
 #pragma unroll
-  for (int o = kLanes / 2; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-  if (live && sub == 0) {
-    seg_key[(int64_t)bh * n_q + pos] = float_order_key(p);
-    if (trace) trace[level * trace_level_stride + (int64_t)bh * n_q + token] = p;
+  for (int o = kLanes / 2; o > 0; o >>= 1)
+#pragma unroll
+    for (int q = 0; q < kProjRows; ++q) p[q] += __shfl_xor_sync(0xffffffffu, p[q], o);
+  if (sub == 0) {
+#pragma unroll
+    for (int q = 0; q < kProjRows; ++q) {
+      if (!live[q]) continue;
+      seg_key[(int64_t)bh * n_q + pos[q]] = float_order_key(p[q]);
+      if (trace) trace[level * trace_level_stride + (int64_t)bh * n_q + token[q]] = p[q];
+    }
   }
 }
 
@@ -806,7 +823,7 @@ static int run_pddp_t(const T* Q, int64_t BH, int n_q, int gs, int32_t* groups, 
           Q, w.perm, n_q, gs, G, level, (int)cpn, w.partials, w.node_mu, w.node_v);
     }
     TLSP_TRY(check_launch());
-    constexpr int kRowsPerBlock = 256 / (D * (int)sizeof(T) / 16);
+    constexpr int kRowsPerBlock = 256 / (D * (int)sizeof(T) / 16) * kProjRows;
     pddp_project_kernel<T, D>
         <<<dim3((unsigned)ceil_div(n_q, kRowsPerBlock), (unsigned)BH), 256, 0, st>>>(
             Q, w.perm, n_q, gs, G, level, w.node_mu, w.node_v, w.seg_key, trace, total);
