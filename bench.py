@@ -16,13 +16,15 @@ fp64 CPU oracle timed on a bounded sample as a reported baseline.
 With --gpus N > 1 (launched by torchrun) rank r runs batch elements
 r*B .. r*B + B - 1 of a global batch of N * B (the path shards by batch with
 no exchange), timings are the max over ranks, and `value` aggregates all
-ranks ("weak" scaling).
+ranks ("weak" scaling); with --shard heads the ranks split the workload's
+heads instead ("strong" scaling: the same job on more GPUs).
 `--impl reference` times the oracle on the host cores instead (rank 0 only).
 """
 from __future__ import annotations
 
 import argparse
 import csv
+import dataclasses
 import io
 import json
 import os
@@ -57,6 +59,9 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--shard", choices=["batch", "heads"], default="batch",
+                    help="multi-GPU split: each rank its own batch element(s) (weak scaling) "
+                         "or the workload's heads split over the ranks (strong scaling)")
     return ap.parse_args()
 
 
@@ -224,8 +229,15 @@ def main():
         return multi.max_over_ranks(info, vals, device=dev)
 
     peaks, peak_kind = load_peaks()
-    # rank r holds batch elements r*B .. r*B + B - 1 of a global batch of world * B
-    it = iter(InputStream(wl, steps=2, batch_offset=multi.batch_offset(wl.batch, rank)))
+    full_wl = wl
+    if args.shard == "heads":
+        # rank r holds its contiguous share of the heads of one fixed batch
+        my_heads = list(multi.head_shard(wl.heads, world, rank))
+        it = iter(InputStream(wl, head_ids=my_heads, steps=2))
+        wl = dataclasses.replace(wl, heads=len(my_heads))
+    else:
+        # rank r holds batch elements r*B .. r*B + B - 1 of a global batch of world * B
+        it = iter(InputStream(wl, steps=2, batch_offset=multi.batch_offset(wl.batch, rank)))
     _, _, Qa, Ka, Va = next(it)
     _, _, Qr, Kr, Vr = next(it)
     Qa, Ka, Va = (t.to(dev) for t in (Qa, Ka, Va))
@@ -315,8 +327,12 @@ def main():
                          statistics.mean(group_ms), statistics.mean(dense_ms),
                          statistics.mean(e2e_ms)])
     total_ms, reuse_mean, anchor_mean, group_mean, dense_mean, e2e_mean = mx
-    flops = wl.reuse_flops()
-    value = multi.aggregate_rate(flops, world, reuse_mean * 1e-3) / 1e12
+    flops = wl.reuse_flops()  # this rank's work
+    # the whole job's work: world copies of the batch shard, or the full workload split by heads
+    strong = args.shard == "heads"
+    job_flops = full_wl.reuse_flops() if strong else world * flops
+    job_dense = full_wl.dense_flops() if strong else world * wl.dense_flops()
+    value = job_flops / (reuse_mean * 1e-3) / 1e12
     peak = float(peaks["bf16_tflops"])
     achieved = flops / (reuse_mean * 1e-3) / 1e12
     traffic = None
@@ -329,20 +345,22 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s (executed, reuse step)",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "strong" if strong else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded smooth field + noise)",
-        "config": dict(config_of(wl), global_batch=world * wl.batch, parallelism=f"dp{world}"),
+        "config": dict(config_of(full_wl),
+                       global_batch=full_wl.batch if strong else world * wl.batch,
+                       parallelism=f"heads{world}" if strong else f"dp{world}"),
         "reuse_ms": reuse_mean, "anchor_ms": anchor_mean, "group_queries_ms": group_mean,
         "dense_pass_ms": dense_mean, "reuse_vs_dense_speedup": dense_mean / reuse_mean,
-        "reuse_dense_equiv_tflops": multi.aggregate_rate(wl.dense_flops(), world,
-                                                         reuse_mean * 1e-3) / 1e12,
+        "reuse_dense_equiv_tflops": job_dense / (reuse_mean * 1e-3) / 1e12,
         "dense_pass_tflops": wl.dense_flops() / (dense_mean * 1e-3) / 1e12,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": "reuse sparse attention (gathered QK^T, PV, +R epilogue)",
                      "peak_kind": f"bf16 dense burst, {peak_kind}",
                      "frac_of_sustained": achieved / float(peaks["bf16_tflops_sustained"])},
-        "e2e": {"value": multi.aggregate_rate(flops, world, e2e_mean * 1e-3) / 1e12,
+        "e2e": {"value": job_flops / (e2e_mean * 1e-3) / 1e12,
                 "unit": "TFLOP/s (executed, reuse step)", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms": e2e_mean},
         "gpu_launches": launches, "clocks": clk,

@@ -56,6 +56,29 @@ def _path_results(wl, stream):
     return out
 
 
+def _path_results_heads(wl, head_ids):
+    """As _path_results, for the given heads of batch element 0 (keys: head ids)."""
+    res = _path_results(wl, InputStream(wl, head_ids=head_ids, steps=2))
+    return {head_ids[h]: v for (b, h), v in res.items()}
+
+
+def _worker_heads(rank, port, out_path):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(WORLD), LOCAL_RANK=str(rank))
+    info = multi.rank_info()
+    multi.init(info, "gloo", timeout_s=60)
+    wl = dataclasses.replace(workload(0), heads=3)  # uneven: 2 heads on rank 0, 1 on rank 1
+    mine = list(multi.head_shard(wl.heads, info.world, info.rank))
+    res = _path_results_heads(wl, mine)
+    gathered = [None] * info.world
+    dist.all_gather_object(gathered, res)
+    multi.barrier(info)
+    if info.is_root:
+        with open(out_path, "wb") as f:
+            pickle.dump(gathered, f)
+    multi.finish(info)
+
+
 def _worker(rank, port, out_path):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
                       WORLD_SIZE=str(WORLD), LOCAL_RANK=str(rank))
@@ -147,3 +170,36 @@ def test_reference_arm_only_on_rank0():
     assert line["impl"] == "reference" and line["n_gpus"] == 2
     assert line["cpu_baseline"]["kind"] == "oracle" and line["value"] > 0
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+
+def test_head_shard_bounds():
+    assert [list(multi.head_shard(12, 5, r)) for r in range(5)] == \
+        [[0, 1, 2], [3, 4, 5], [6, 7], [8, 9], [10, 11]]
+    assert list(multi.head_shard(40, 8, 7)) == list(range(35, 40))
+    for heads, world in ((12, 8), (40, 8), (3, 2), (7, 7)):
+        got = [h for r in range(world) for h in multi.head_shard(heads, world, r)]
+        assert got == list(range(heads))
+    with pytest.raises(ValueError):
+        multi.head_shard(3, 4, 0)
+    with pytest.raises(ValueError):
+        multi.head_shard(8, 2, 2)
+
+
+def test_head_shards_equal_unsharded_heads(tmp_path):
+    """Heads split over two gloo ranks: every head's grouping, selection, residual and
+    reuse output equal the unsharded run's for that head."""
+    out = str(tmp_path / "heads.pkl")
+    mp.start_processes(_worker_heads, args=(_free_port(), out), nprocs=WORLD, join=True,
+                       start_method="spawn")
+    with open(out, "rb") as f:
+        gathered = pickle.load(f)
+    wl = dataclasses.replace(workload(0), heads=3)
+    ref = _path_results_heads(wl, list(range(wl.heads)))
+    seen = {}
+    for res in gathered:
+        seen.update(res)
+    assert sorted(seen) == list(range(wl.heads))
+    for h, v in seen.items():
+        for key in ("Q", "groups", "idx", "R", "O"):
+            assert np.array_equal(v[key], ref[h][key]), (h, key)

@@ -5,7 +5,9 @@ exact group scores, the top-k selection and both sparse passes are defined
 per head (MC-Sparse review, section 3: groups, scores and the cached
 selection belong to one head's attention). A job of `world * B` batch
 elements therefore gives rank r the elements [r*B, (r+1)*B) and runs them
-with no exchange of data between ranks. The only collectives are the ones a
+with no exchange of data between ranks (weak scaling); alternatively the
+heads of a fixed batch are split over the ranks (`head_shard`, strong
+scaling). The only collectives are the ones a
 measurement needs: a barrier around the timed region and a max over ranks of
 the measured times.
 """
@@ -52,6 +54,19 @@ def shard_bounds(global_batch: int, world: int, rank: int) -> range:
         raise ValueError(f"cannot shard a batch of {global_batch} over {world} ranks")
     per = global_batch // world
     return range(batch_offset(per, rank), batch_offset(per, rank) + per)
+
+
+def head_shard(heads: int, world: int, rank: int) -> range:
+    """Heads of `rank` when one batch element's heads are split over the ranks
+    (contiguous, as equal as possible: the first heads % world ranks hold one
+    more). Grouping, scores, selection and both sparse passes are per head, so
+    the shards need no exchange either; this splits a fixed problem (strong
+    scaling) where batch sharding grows it (weak scaling)."""
+    if world < 1 or not 0 <= rank < world or heads < world:
+        raise ValueError(f"cannot split {heads} heads over {world} ranks")
+    base, extra = divmod(heads, world)
+    start = rank * base + min(rank, extra)
+    return range(start, start + base + (1 if rank < extra else 0))
 
 
 def init(info: RankInfo, backend: str, device=None, timeout_s: float = 120.0) -> None:
