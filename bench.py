@@ -206,7 +206,6 @@ def main():
     from token_level_sparse_pddp_b200.synthetic import InputStream, workload
     wl = workload(args.workload)
     if args.heads:
-        import dataclasses
         wl = dataclasses.replace(wl, heads=args.heads, name=f"{wl.name}-H{args.heads}")
     if args.impl == "reference":
         os.environ.setdefault("OMP_NUM_THREADS", str(os.cpu_count() or 1))
