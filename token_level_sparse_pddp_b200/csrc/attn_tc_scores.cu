@@ -14,14 +14,13 @@
 // no cross-thread reduction and no atomics; the per-query LSE (in log2 units)
 // is a shared-memory broadcast. S^T is double-buffered in TMEM so the next
 // chunk's MMA runs while a chunk is summed.
-// Warp roles (416 threads): warps 0-3 and 4-7 sum (lane t of both warps w
-// and w + 4 is key j0 + 32 (w % 4) + t; warps 0-3 take the group's query
-// columns 0-63 and warps 4-7 columns 64-127, so two warps per SM sub-partition
-// hide each other's TMEM and SFU latency); warps 4-7 hand their partial sums
-// to warps 0-3 through a double-buffered shared-memory slot, and warps 0-3
-// store the total. Warps 8-11 gather Q_g with 16-byte cp.async (128-byte
-// swizzle), then lane 0 of warp 8 issues the K loads; warp 12 allocates TMEM
-// and lane 0 issues tcgen05.mma.
+// Warp roles (416 threads): warps 0-3 sum the even chunks (TMEM buffer 0)
+// and warps 4-7 the odd ones (buffer 1), each lane over all 128 query
+// columns of its key, so the two warps of an SM sub-partition work on
+// different chunks and one's TMEM loads overlap the other's exp2; each
+// warpgroup stores its chunk's sums itself. Warps 8-11 gather Q_g with
+// 16-byte cp.async (128-byte swizzle), then lane 0 of warp 8 issues the K
+// loads; warp 12 allocates TMEM and lane 0 issues tcgen05.mma.
 // Every wait is bounded (1 s); on expiry the kernel records TLSP_ERR_TIMEOUT
 // and unwinds.
 #include "kernels.h"
@@ -39,8 +38,7 @@ constexpr int kKSlots = 4;
 constexpr uint32_t kSmQ = 0, kSmK = kTileBytes;
 constexpr uint32_t kSmBar = (1 + kKSlots) * kTileBytes;
 constexpr uint32_t kSmLse = kSmBar + 256;
-constexpr uint32_t kSmX = kSmLse + kTile * 4;  // partial sums, 2 x 128 floats
-constexpr uint32_t kSmemBytes = kSmX + 2 * kTile * 4 + 1024;
+constexpr uint32_t kSmemBytes = kSmLse + kTile * 4 + 1024;
 constexpr uint32_t kTmCols = 256;
 constexpr uint64_t kWaitNs = 1000000000ull;
 
@@ -48,7 +46,6 @@ struct Bars {
   uint64_t q_full;
   uint64_t k_full[kKSlots], k_empty[kKSlots];
   uint64_t s_full[2], s_empty[2];
-  uint64_t x_full[2], x_empty[2];  // partial sums of warps 4-7 -> warps 0-3
   uint64_t drain;
   uint32_t tmem_base;
   int abort;
@@ -100,9 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&bars.s_full[s], 1);
-      ptx::mbar_init(&bars.s_empty[s], 256);
-      ptx::mbar_init(&bars.x_full[s], 128);
-      ptx::mbar_init(&bars.x_empty[s], 128);
+      ptx::mbar_init(&bars.s_empty[s], 128);
     }
     ptx::mbar_init(&bars.drain, 1);
     bars.abort = 0;
@@ -196,60 +191,55 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp < 8) {
     // ------------------------------------------------------------ sums
-    const int r = tid & 127, half = warp >> 2;  // key lane r, query columns 64*half ..
-    float* xs = reinterpret_cast<float*>(smem + kSmX);
-    if (half == 0) {
+    // warpgroup h = warp / 4 takes the chunks j = h, h + 2, ... (TMEM buffer h);
+    // lane r of warp w is key j * 128 + 32 (w % 4) + r and sums all 128 columns
+    const int r = tid & 127, h = warp >> 2;
+    if (h == 0) {
       // log2-unit LSE of the group's queries; padding rows contribute exp2(-inf) = 0
       const int tok = r < p.gs ? grp[r] : -1;
       lse2_s[r] = (tok >= 0 && tok < p.n_q) ? p.lse[bh * p.n_q + tok] * 1.4426950408889634f
                                              : INFINITY;
     }
     asm volatile("bar.sync 2, 256;" ::: "memory");
-    float lse2[64];
-#pragma unroll
-    for (int e = 0; e < 64; ++e) lse2[e] = lse2_s[64 * half + e];
-    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16) + 64 * half;
+    const float4* l4 = reinterpret_cast<const float4*>(lse2_s);
+    const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16) + h * kTile;
     float* out = p.S + (bh * p.G + g) * (int64_t)p.n_kv;
-    for (int j = 0; j < n_chunks; ++j) {
-      const int s = j & 1;
-      if (!ptx::mbar_wait(&bars.s_full[s], (j >> 1) & 1, abort_flag, kWaitNs)) {
+    for (int j = h; j < n_chunks; j += 2) {
+      if (!ptx::mbar_wait(&bars.s_full[h], (j >> 1) & 1, abort_flag, kWaitNs)) {
         fail(bars, p.status);
         break;
       }
       ptx::tc_fence_after();
       float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      // columns 32q .. 32q + 31 of this lane against the queries' LSE
+      auto sum32 = [&](const uint32_t (&c)[32], int q) {
+#pragma unroll
+        for (int e = 0; e < 32; e += 4) {
+          const float4 l = l4[(32 * q + e) >> 2];
+          acc[0] += ptx::ex2(fmaf(__uint_as_float(c[e + 0]), p.scale_log2, -l.x));
+          acc[1] += ptx::ex2(fmaf(__uint_as_float(c[e + 1]), p.scale_log2, -l.y));
+          acc[2] += ptx::ex2(fmaf(__uint_as_float(c[e + 2]), p.scale_log2, -l.z));
+          acc[3] += ptx::ex2(fmaf(__uint_as_float(c[e + 3]), p.scale_log2, -l.w));
+        }
+      };
+      // each quarter's TMEM load is in flight while the one before it is summed
       uint32_t c0[32], c1[32];
-      ptx::tmem_ld32(tl + s * kTile, c0);
-      ptx::tmem_ld32(tl + s * kTile + 32, c1);
+      ptx::tmem_ld32(tl, c0);
       ptx::tmem_ld_wait(c0);
-      ptx::reg_barrier(c1);
+      ptx::tmem_ld32(tl + 32, c1);
+      sum32(c0, 0);
+      ptx::tmem_ld_wait(c1);
+      ptx::tmem_ld32(tl + 64, c0);
+      sum32(c1, 1);
+      ptx::tmem_ld_wait(c0);
+      ptx::tmem_ld32(tl + 96, c1);
+      sum32(c0, 2);
+      ptx::tmem_ld_wait(c1);
       ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars.s_empty[s]);  // S is in registers: the MMA may overwrite it
-#pragma unroll
-      for (int e = 0; e < 32; ++e)
-        acc[e & 3] += ptx::ex2(fmaf(__uint_as_float(c0[e]), p.scale_log2, -lse2[e]));
-#pragma unroll
-      for (int e = 0; e < 32; ++e)
-        acc[e & 3] += ptx::ex2(fmaf(__uint_as_float(c1[e]), p.scale_log2, -lse2[32 + e]));
-      const float part = (acc[0] + acc[1]) + (acc[2] + acc[3]);
-      if (half == 1) {
-        // slot s is free once warps 0-3 have read it for chunk j - 2
-        if (j >= 2 && !ptx::mbar_wait(&bars.x_empty[s], ((j >> 1) - 1) & 1, abort_flag, kWaitNs)) {
-          fail(bars, p.status);
-          break;
-        }
-        xs[s * kTile + r] = part;
-        ptx::mbar_arrive(&bars.x_full[s]);
-      } else {
-        if (!ptx::mbar_wait(&bars.x_full[s], (j >> 1) & 1, abort_flag, kWaitNs)) {
-          fail(bars, p.status);
-          break;
-        }
-        const float total = part + xs[s * kTile + r];
-        ptx::mbar_arrive(&bars.x_empty[s]);
-        const int key = j * kTile + r;
-        if (key < p.n_kv) out[key] = total;
-      }
+      ptx::mbar_arrive(&bars.s_empty[h]);  // S is in registers: the MMA may overwrite it
+      sum32(c1, 3);
+      const int key = j * kTile + r;
+      if (key < p.n_kv) out[key] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
     }
   }
 
