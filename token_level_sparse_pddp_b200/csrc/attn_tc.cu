@@ -1,6 +1,6 @@
-// Attention on the sm_100a tensor cores (bf16, head_dim 128): the dense pass
-// of the anchor step and the gathered sparse pass of anchor and reuse steps,
-// with the dense-sparse residual fused into the sparse epilogue.
+// Sparse attention on the sm_100a tensor cores (bf16, head_dim 128): the
+// gathered pass of anchor and reuse steps, with the dense-sparse residual
+// fused into the epilogue (the dense pass is in attn_tc_dense.cu).
 //
 // MC-Sparse review, section 3: the anchor step runs dense attention (its
 // output and the exact scores), each query group attends only to its own
@@ -8,19 +8,17 @@
 // stores R = O_full - O_sparse and the reuse steps return O_sparse + R
 // (additive correction for the discarded tail).
 //
-// One CTA per 128-query tile: a block of 128 consecutive queries (dense) or
-// a group's queries (sparse; g_s <= 128 is one tile, padding rows are zero and
-// never written back). Warp roles (416 threads, one CTA per SM):
+// One CTA per 128-query tile of a group (g_s <= 128 is one tile; padding
+// rows are zero and never written back). Warp roles (416 threads, one CTA
+// per SM):
 //   warps 0-3  softmax + epilogue: thread t owns query row t = TMEM lane t;
-//   warps 4-11 producers. Dense: lane 0 of warp 4 loads the Q tile and the K
-//              and V tiles of each chunk of 128 keys with TMA box loads.
-//              Sparse: together they load the tile's selection into shared
-//              memory and gather its Q rows, then warps 4-7 gather the K rows
-//              and warps 8-11 the V rows of each chunk of 128 selected keys,
-//              with 16-byte cp.async (eight issuing warps: the gather rate
-//              grows with the warps that issue, not only with the bytes in
-//              flight). Either way the tiles land in 128-byte swizzled shared
-//              memory (the tcgen05 canonical layout);
+//   warps 4-11 producers: together they load the tile's selection into
+//              shared memory and gather its Q rows, then warps 4-7 gather the
+//              K rows and warps 8-11 the V rows of each chunk of 128 selected
+//              keys, with 16-byte cp.async (eight issuing warps: the gather
+//              rate grows with the warps that issue, not only with the bytes
+//              in flight), into 128-byte swizzled shared memory (the tcgen05
+//              canonical layout);
 //   warp 12    allocates TMEM; lane 0 issues the tcgen05.mma instructions.
 // Per chunk j: S_j = Q K_j^T (M=N=K=128, fp32 in TMEM), online softmax with
 // exp2 on the SFU (S read from TMEM 64 columns at a time, the second half
@@ -31,20 +29,19 @@
 // shared-memory slots and V two, so loads run ahead of the math.
 // The softmax keeps a reference max per row and computes each chunk in one
 // pass against it; only when a chunk's max exceeds the reference by more than
-// 2^8 is the reference raised, O rescaled in TMEM and the chunk recomputed.
+// 2^8 is the reference raised, O rescaled in TMEM and the chunk recomputed
+// (by the whole warp: its TMEM accesses are warp-collective).
 // Between raises the stale reference is used for numerator and denominator
 // alike, which cancels exactly in O / l.
 // Every wait is bounded (1 s); on expiry the kernel records
 // TLSP_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
-#include <algorithm>
-
 #include "kernels.h"
 #include "tc_ptx.cuh"
 
 namespace tlsp {
 namespace {
 
-enum Mode { kDense = 0, kAnchor = 1, kReuse = 2 };
+enum Mode { kAnchor = 1, kReuse = 2 };
 
 constexpr int kTile = 128;
 constexpr int kD = 128;
@@ -75,19 +72,17 @@ struct Bars {
 static_assert(sizeof(Bars) <= 256, "barrier block");
 
 struct AttnParams {
-  CUtensorMap tmQ, tmK, tmV;  // dense: [BH*n, 128] bf16 row maps, box 64 x 128, 128-byte swizzle
   const __nv_bfloat16* __restrict__ Q;
   const __nv_bfloat16* __restrict__ K;
   const __nv_bfloat16* __restrict__ V;
   const int32_t* __restrict__ groups;
   const int32_t* __restrict__ indices;
-  int n_q, n_kv, gs, G, k, tiles_per_group, q_tiles;
+  int n_q, n_kv, gs, G, k, tiles_per_group;
   float scale_log2;
   const __nv_bfloat16* __restrict__ O_full;  // anchor: the dense output as stored
   float* __restrict__ R_out;                 // anchor
   const float* __restrict__ R_in;            // reuse
-  __nv_bfloat16* __restrict__ O_out;         // dense and reuse
-  float* __restrict__ lse;                   // dense: [BH, n_q] natural-log partition
+  __nv_bfloat16* __restrict__ O_out;         // reuse
   int wave;                                  // CTAs resident at once (one per SM)
   int* status;
 };
@@ -184,7 +179,6 @@ __device__ __forceinline__ void fail(Bars& b, int* status) {
 template <int kMode>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(const __grid_constant__ AttnParams p) {
-  constexpr bool kSparse = kMode != kDense;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = ptx::smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -193,26 +187,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = &bars.abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  // tile -> (head, rows): sparse tiles are (group, 128-row part of the group),
-  // dense tiles are blocks of 128 consecutive queries
-  const int tiles_per_head = kSparse ? p.G * p.tiles_per_group : p.q_tiles;
+  // tile -> (head, group, 128-row part of the group)
+  const int tiles_per_head = p.G * p.tiles_per_group;
   const int64_t bh = blockIdx.x / tiles_per_head;
   const int rem = blockIdx.x % tiles_per_head;
-  const int g = kSparse ? rem / p.tiles_per_group : 0;
-  const int t = kSparse ? rem % p.tiles_per_group : rem;
-  const int32_t* grp = kSparse ? p.groups + (bh * p.G + g) * (int64_t)p.gs : nullptr;
-  const int32_t* sel = kSparse ? p.indices + (bh * p.G + g) * (int64_t)p.k : nullptr;
-  const int n_keys = kSparse ? p.k : p.n_kv;
+  const int g = rem / p.tiles_per_group;
+  const int t = rem % p.tiles_per_group;
+  const int32_t* grp = p.groups + (bh * p.G + g) * (int64_t)p.gs;
+  const int32_t* sel = p.indices + (bh * p.G + g) * (int64_t)p.k;
+  const int n_keys = p.k;
   const int n_chunks = (n_keys + kTile - 1) / kTile;
 
   if (tid == 0) {
-    ptx::mbar_init(&bars.q_full, kSparse ? 256 : 1);
+    ptx::mbar_init(&bars.q_full, 256);
     for (int s = 0; s < kKSlots; ++s) {
-      ptx::mbar_init(&bars.k_full[s], kSparse ? 128 : 1);
+      ptx::mbar_init(&bars.k_full[s], 128);
       ptx::mbar_init(&bars.k_empty[s], 1);
     }
     for (int s = 0; s < kVSlots; ++s) {
-      ptx::mbar_init(&bars.v_full[s], kSparse ? 128 : 1);
+      ptx::mbar_init(&bars.v_full[s], 128);
       ptx::mbar_init(&bars.v_empty[s], 1);
     }
     for (int s = 0; s < 2; ++s) {
@@ -234,49 +227,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
 
-  if (!kSparse && warp == 4) {
-    // ------------------------------------------------------------ dense producer
-    if (lane == 0) {
-      const int q_row = (int)(bh * p.n_q) + t * kTile, kv_row = (int)(bh * p.n_kv);
-      ptx::mbar_arrive_expect_tx(&bars.q_full, kTileBytes);
-      ptx::tma_load_2d(base + kSmQ, &p.tmQ, 0, q_row, &bars.q_full);
-      ptx::tma_load_2d(base + kSmQ + kHalfBytes, &p.tmQ, 64, q_row, &bars.q_full);
-      int issued_k = 0, issued_v = 0;
-      bool ok = true;
-      for (int j = 0; j < n_chunks; ++j) {
-        const int ks = j % kKSlots, ku = j / kKSlots, vs = j % kVSlots, vu = j / kVSlots;
-        const int y = kv_row + j * kTile;
-        if (ku > 0 && !ptx::mbar_wait(&bars.k_empty[ks], (ku - 1) & 1, abort_flag, kWaitNs)) {
-          ok = false;
-          break;
-        }
-        ptx::mbar_arrive_expect_tx(&bars.k_full[ks], kTileBytes);
-        ptx::tma_load_2d(base + kSmK + ks * kTileBytes, &p.tmK, 0, y, &bars.k_full[ks]);
-        ptx::tma_load_2d(base + kSmK + ks * kTileBytes + kHalfBytes, &p.tmK, 64, y,
-                         &bars.k_full[ks]);
-        issued_k = j + 1;
-        if (vu > 0 && !ptx::mbar_wait(&bars.v_empty[vs], (vu - 1) & 1, abort_flag, kWaitNs)) {
-          ok = false;
-          break;
-        }
-        ptx::mbar_arrive_expect_tx(&bars.v_full[vs], kTileBytes);
-        ptx::tma_load_2d(base + kSmV + vs * kTileBytes, &p.tmV, 0, y, &bars.v_full[vs]);
-        ptx::tma_load_2d(base + kSmV + vs * kTileBytes + kHalfBytes, &p.tmV, 64, y,
-                         &bars.v_full[vs]);
-        issued_v = j + 1;
-      }
-      if (!ok) {
-        fail(bars, p.status);
-        // loads already issued land before the CTA's shared memory goes away
-        for (int j = max(0, issued_k - kKSlots); j < issued_k; ++j)
-          ptx::mbar_wait(&bars.k_full[j % kKSlots], (j / kKSlots) & 1, nullptr, kWaitNs);
-        for (int j = max(0, issued_v - kVSlots); j < issued_v; ++j)
-          ptx::mbar_wait(&bars.v_full[j % kVSlots], (j / kVSlots) & 1, nullptr, kWaitNs);
-        ptx::mbar_wait(&bars.q_full, 0, nullptr, kWaitNs);
-      }
-    }
-    __syncwarp();
-  } else if (kSparse && warp >= 4 && warp < 12) {
+  if (warp >= 4 && warp < 12) {
     // ------------------------------------------------------------ producers
     const int pt = tid - 128;
     // The tile's selection goes to shared memory once (4-byte cp.async by all
@@ -391,23 +342,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ softmax
     const int r = tid;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    int tok;
-    if (kSparse) {
-      const int gr = t * kTile + r;
-      tok = gr < p.gs ? grp[gr] : -1;
-      if (tok >= p.n_q) tok = -1;
-      if (tok >= 0) {  // the row the epilogue reads, towards L2 while the tile computes
-        const int64_t row = (bh * p.n_q + tok) * kD;
-        if (kMode == kReuse) {
+    const int gr = t * kTile + r;
+    int tok = gr < p.gs ? grp[gr] : -1;
+    if (tok >= p.n_q) tok = -1;
+    if (tok >= 0) {  // the row the epilogue reads, towards L2 while the tile computes
+      const int64_t row = (bh * p.n_q + tok) * kD;
+      if (kMode == kReuse) {
 #pragma unroll
-          for (int l = 0; l < 4; ++l) prefetch_l2(p.R_in + row + 32 * l);
-        } else {
-          prefetch_l2(p.O_full + row);
-          prefetch_l2(p.O_full + row + 64);
-        }
+        for (int l = 0; l < 4; ++l) prefetch_l2(p.R_in + row + 32 * l);
+      } else {
+        prefetch_l2(p.O_full + row);
+        prefetch_l2(p.O_full + row + 64);
       }
-    } else {
-      tok = t * kTile + r < p.n_q ? t * kTile + r : -1;
     }
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
@@ -474,7 +420,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool raise = (j == 0);
       if (!raise) {
         p_pass(m_run, sum, mx);  // speculative: usually the reference max still holds
-        raise = mx * p.scale_log2 > m_run + kRescaleLog2;
+        // the rescale below is made of warp-collective TMEM accesses, so the
+        // warp takes it together when any of its rows needs it
+        raise = __any_sync(0xffffffffu, mx * p.scale_log2 > m_run + kRescaleLog2);
       } else {
         // first chunk: its max becomes the reference
         float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -490,7 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mx = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
       }
       if (raise) {
-        const float m_tile = mx * p.scale_log2;
+        // rows of the warp that do not need it keep their reference (factor 1)
+        const float m_tile = j > 0 ? fmaxf(mx * p.scale_log2, m_run) : mx * p.scale_log2;
         if (j > 0) {
           // raise the reference max: O *= 2^(m_run - m_tile) once PV(j-1) has landed
           const float f = ptx::ex2(m_run - m_tile);
@@ -523,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Epilogue operands (R rows for the reuse step, O_full rows for the anchor
     // step) are read one 32-column block ahead: block 0 before the final wait,
     // block q + 1 while block q's TMEM load is in flight.
-    const bool has_row = kMode != kDense && tok >= 0;
+    const bool has_row = tok >= 0;
     float4 rb[2][8];  // reuse: R, 32 fp32 columns per block
     uint4 ob[2][4];   // anchor: O_full, 32 bf16 columns per block
     auto load_block = [&](int q, int b) {
@@ -544,8 +493,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
       ptx::tc_fence_after();
       const float inv = 1.f / l_run;
-      if (kMode == kDense && tok >= 0)  // log partition in natural units: (m + log2 l) ln 2
-        p.lse[bh * p.n_q + tok] = (m_run + __log2f(l_run)) * 0.6931471805599453f;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t o[32];
@@ -619,7 +566,6 @@ AttnParams base_params(const AttnArgs& a) {
   p.G = a.G;
   p.k = a.k;
   p.tiles_per_group = (a.gs + kTile - 1) / kTile;
-  p.q_tiles = (a.n_q + kTile - 1) / kTile;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
   p.status = a.status;
   int dev = 0, sms = 0;
@@ -649,21 +595,6 @@ int tc_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices,
     launch<kAnchor>(p, tiles, st);
   else
     launch<kReuse>(p, tiles, st);
-  return check_launch();
-}
-
-int tc_dense(const AttnArgs& a, void* O, float* lse, cudaStream_t st) {
-  AttnParams p = base_params(a);
-  if ((uint64_t)a.BH * (uint64_t)std::max(a.n_q, a.n_kv) >= 0x7fffffffull)
-    return TLSP_ERR_UNSUPPORTED;
-  TLSP_TRY(make_tmap_bf16_rows(&p.tmQ, a.Q, (uint64_t)a.BH * a.n_q, kD, 64, kTile));
-  TLSP_TRY(make_tmap_bf16_rows(&p.tmK, a.K, (uint64_t)a.BH * a.n_kv, kD, 64, kTile));
-  TLSP_TRY(make_tmap_bf16_rows(&p.tmV, a.V, (uint64_t)a.BH * a.n_kv, kD, 64, kTile));
-  p.O_out = (__nv_bfloat16*)O;
-  p.lse = lse;
-  const int64_t tiles = a.BH * p.q_tiles;
-  if (tiles > 0x7fffffffLL) return TLSP_ERR_UNSUPPORTED;
-  launch<kDense>(p, tiles, st);
   return check_launch();
 }
 

@@ -57,11 +57,12 @@ int simt_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices
 int make_tmap_bf16_rows(CUtensorMap* map, const void* ptr, uint64_t rows, uint64_t cols,
                         uint32_t box_cols, uint32_t box_rows);
 
-// attn_tc.cu: tensor-core dense pass and gathered sparse pass (bf16, d = 128)
+// attn_tc.cu: tensor-core gathered sparse pass (bf16, d = 128)
 bool tc_attention_supported(const AttnArgs& a);
 int tc_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices,
               const void* O_full, float* R_out, const float* R_in, void* O_out,
               cudaStream_t st);
+// attn_tc_dense.cu: tensor-core dense pass (same support condition)
 int tc_dense(const AttnArgs& a, void* O, float* lse, cudaStream_t st);
 
 // attn_tc_scores.cu: exact group scores on the tensor cores (bf16, d = 128, g_s <= 128)
