@@ -17,8 +17,6 @@ import torch
 from oracle import oracle as orc
 from tests.parity import TOL
 
-pytestmark = pytest.mark.gpu
-
 N_Q, N_KV, D, H = 256, 552, 128, 2  # 2 query tiles; 4 full key chunks + a ragged one
 # (key, channel, rows, key value): those rows get q[channel] = 8, so their logit on
 # the key is 8 * value / sqrt(128) nats, 28-42 nats above everything else
@@ -49,6 +47,42 @@ def _inputs():
     return Q.bfloat16(), K.bfloat16(), V.bfloat16()
 
 
+def _log2_logits(Q, K):
+    """fp64 logits of the bf16 inputs in log2 units, [H, n_q, n_kv]."""
+    q, k = Q[0].double().numpy(), K[0].double().numpy()
+    return np.einsum("hqd,hkd->hqk", q, k) / np.sqrt(D) / np.log(2.0)
+
+
+def test_inputs_raise_in_part_of_each_warp():
+    """The inputs do what the GPU tests need: in the dense pass (chunks of 128 keys
+    in order) and in the sparse pass (the selection below), some rows of a warp
+    exceed their running reference by more than 2^8 in a later chunk while other
+    rows of the same warp do not."""
+    Q, K, _ = _inputs()
+    x = _log2_logits(Q, K)
+    sel = np.union1d(np.arange(0, N_KV, 2), np.arange(1, 217, 2))
+    for keys in (np.arange(N_KV), sel):
+        xs = x[:, :, keys]
+        ref = xs[:, :, :128].max(axis=2)          # reference after the first chunk
+        mixed = 0
+        for c0 in range(128, keys.shape[0], 128):
+            cm = xs[:, :, c0:c0 + 128].max(axis=2)
+            raise_ = cm > ref + 8.0
+            for w in range(N_Q // 32):
+                rows = slice(32 * w, 32 * (w + 1))
+                r = raise_[:, rows]
+                mixed += int((r.any(axis=1) & ~r.all(axis=1)).sum())
+                # a warp that raises moves every row's reference to max(ref, chunk max)
+                ref[:, rows] = np.where(r.any(axis=1, keepdims=True),
+                                        np.maximum(ref[:, rows], cm[:, rows]), ref[:, rows])
+        assert mixed > 0
+    # and inside the first chunk, after its first 32-column block, for some rows only
+    first = x[:, :, :128]
+    late = first[:, :, 32:].max(axis=2) > first[:, :, :32].max(axis=2) + 8.0
+    assert late.any() and not late.all()
+
+
+@pytest.mark.gpu
 def test_dense_partial_warp_raises(T):
     Q, K, V = _inputs()
     Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
@@ -70,6 +104,7 @@ def test_dense_partial_warp_raises(T):
         assert np.abs(lse[0, h] - L).max() <= 1e-3, (h, np.abs(lse[0, h] - L).max())
 
 
+@pytest.mark.gpu
 def test_sparse_partial_warp_raises(T):
     """The gathered pass over a selection that holds the spike keys in its chunks
     0-2 (positions 70, 222, 258, 333)."""
