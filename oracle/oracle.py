@@ -249,3 +249,67 @@ def pooled_block_scores(Qg, K, b: int) -> np.ndarray:
 def pooled_block_select(Qg, K, k: int, b: int) -> np.ndarray:
     """Block-sparse baseline selection: k / b blocks by mean-pooled score, expanded."""
     return select_blocks(pooled_block_scores(Qg, K, b), k // b, b)
+
+
+# ----------------------------------------------------------------- error decomposition
+# The review's account of the dense-sparse gap (section 2 and its Fig. 2): the
+# sparse output differs from dense attention through the discarded tail (keys
+# left out even by an exact per-query selection), structural binding (one
+# selection shared by a query group, or by a key block) and selection error
+# (approximate scores). Each rung below is one selection; its error is the
+# relative L2 distance of the fp64 sparse output to the fp64 dense output.
+
+def sparse_output(Q, K, V, groups, gs: int, idx) -> np.ndarray:
+    """Sparse attention of every query of every head over its group's selection.
+
+    Q [B, H, n_q, d], K, V [B, H, n_kv, d], groups [B, H, G*gs] (-1 padding),
+    idx [B, H, G, k] -> O [B, H, n_q, d] in fp64 (no residual)."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    groups, idx = np.asarray(groups), np.asarray(idx)
+    B, H, n_q, d = Q.shape
+    O = np.zeros((B, H, n_q, d))
+    G = -(-n_q // gs)
+    for b in range(B):
+        for h in range(H):
+            for g in range(G):
+                rows = group_rows(groups[b, h], gs, g)
+                if rows.size:
+                    O[b, h, rows] = sparse(Q[b, h][rows], K[b, h], V[b, h], idx[b, h, g])
+    return O
+
+
+def dense_output(Q, K, V) -> np.ndarray:
+    """Dense attention of every query of every head -> O [B, H, n_q, d] in fp64."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    O = np.empty(Q.shape)
+    for b in range(Q.shape[0]):
+        for h in range(Q.shape[1]):
+            O[b, h], _ = dense(Q[b, h], K[b, h], V[b, h])
+    return O
+
+
+def rel_l2(O, O_ref) -> float:
+    """|O - O_ref| / |O_ref| over the whole tensor."""
+    O, O_ref = _f64(O), _f64(O_ref)
+    return float(np.linalg.norm(O - O_ref) / np.linalg.norm(O_ref))
+
+
+def rel_l2_head_mean(O, O_ref) -> float:
+    """Mean over (batch, head) of each head's relative L2 distance."""
+    O, O_ref = _f64(O), _f64(O_ref)
+    B, H = O.shape[:2]
+    a, r = O.reshape(B, H, -1), O_ref.reshape(B, H, -1)
+    return float((np.linalg.norm(a - r, axis=2) / np.linalg.norm(r, axis=2)).mean())
+
+
+def decomposition(Q, K, V, rungs):
+    """Errors of a ladder of selections against dense attention, in fp64.
+
+    rungs: list of (groups [B, H, G*gs], gs, idx [B, H, G, k]) -> list of
+    (rel_l2, rel_l2_head_mean), one per rung, in order."""
+    O_dense = dense_output(Q, K, V)
+    out = []
+    for groups, gs, idx in rungs:
+        O = sparse_output(Q, K, V, groups, gs, idx)
+        out.append((rel_l2(O, O_dense), rel_l2_head_mean(O, O_dense)))
+    return out

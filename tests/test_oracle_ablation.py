@@ -70,3 +70,75 @@ def test_block_selection_with_all_keys_gives_dense_attention():
     assert np.array_equal(idx, np.arange(24))
     O, _ = orc.dense(Q, K, V)
     assert np.allclose(orc.sparse(Q, K, V, idx), O, rtol=1e-13, atol=1e-13)
+
+
+# ----------------------------------------------------------------- error decomposition
+
+def _textbook_sparse_row(q, K, V, sel):
+    """Softmax of q . K[sel] / sqrt(d) over the selected keys only, times V[sel]."""
+    s = K[sel] @ q / np.sqrt(q.shape[0])
+    p = np.exp(s - s.max())
+    return (p / p.sum()) @ V[sel]
+
+
+def test_rel_l2_closed_forms():
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((2, 3, 5, 4))
+    assert orc.rel_l2(x, x) == 0.0 and orc.rel_l2_head_mean(x, x) == 0.0
+    assert abs(orc.rel_l2(2 * x, x) - 1.0) < 1e-12
+    assert abs(orc.rel_l2_head_mean(-x, x) - 2.0) < 1e-12
+    y = x.copy()
+    y[1, 2] *= 3.0   # one head off by 2x its own norm
+    assert abs(orc.rel_l2_head_mean(y, x) - 2.0 / 6) < 1e-12
+
+
+def test_sparse_output_all_keys_is_dense_output():
+    rng = np.random.default_rng(7)
+    B, H, n, d, gs = 1, 2, 12, 8, 4
+    Q, K, V = (rng.standard_normal((B, H, n, d)) for _ in range(3))
+    groups = np.broadcast_to(orc.raster_groups(n, gs), (B, H, n)).copy()
+    idx = np.broadcast_to(np.arange(n, dtype=np.int32), (B, H, n // gs, n)).copy()
+    O_sp = orc.sparse_output(Q, K, V, groups, gs, idx)
+    assert np.abs(O_sp - orc.dense_output(Q, K, V)).max() < 1e-12
+    err = orc.decomposition(Q, K, V, [(groups, gs, idx)])
+    assert err[0][0] < 1e-12 and err[0][1] < 1e-12
+
+
+def test_sparse_output_matches_textbook_per_group():
+    """Ragged grouping in a shuffled order, a different selection per group."""
+    rng = np.random.default_rng(8)
+    B, H, n, d, gs, k = 2, 1, 10, 6, 4, 5
+    Q, K, V = (rng.standard_normal((B, H, n, d)) for _ in range(3))
+    G = -(-n // gs)
+    groups = np.full((B, H, G * gs), -1, dtype=np.int32)
+    idx = np.empty((B, H, G, k), dtype=np.int32)
+    for b in range(B):
+        perm = rng.permutation(n)
+        for g in range(G):
+            members = np.sort(perm[g * gs:(g + 1) * gs])
+            groups[b, 0, g * gs:g * gs + members.size] = members
+            idx[b, 0, g] = np.sort(rng.choice(n, size=k, replace=False))
+    O = orc.sparse_output(Q, K, V, groups, gs, idx)
+    for b in range(B):
+        for g in range(G):
+            for t in orc.group_rows(groups[b, 0], gs, g):
+                want = _textbook_sparse_row(Q[b, 0, t], K[b, 0], V[b, 0], idx[b, 0, g])
+                assert np.abs(O[b, 0, t] - want).max() < 1e-12
+
+
+def test_decomposition_per_query_selection_by_hand():
+    """One query, two keys of three: the error is computed by hand from the
+    textbook dense and sparse outputs."""
+    q = np.array([[[[1.0, 0.0]]]])
+    K = np.array([[[[1.0, 0.0], [0.0, 1.0], [-1.0, 0.0]]]])
+    V = np.array([[[[1.0, 0.0], [0.0, 1.0], [0.0, 0.0]]]])
+    s = np.array([1.0, 0.0, -1.0]) / np.sqrt(2)
+    p = np.exp(s) / np.exp(s).sum()
+    dense = p @ V[0, 0]
+    p2 = np.exp(s[:2]) / np.exp(s[:2]).sum()
+    sparse = p2 @ V[0, 0, :2]
+    want = np.linalg.norm(sparse - dense) / np.linalg.norm(dense)
+    groups = np.zeros((1, 1, 1), dtype=np.int32)
+    idx = np.array([[[[0, 1]]]], dtype=np.int32)
+    (got, got_h), = orc.decomposition(q, K, V, [(groups, 1, idx)])
+    assert abs(got - want) < 1e-12 and abs(got_h - want) < 1e-12
