@@ -59,6 +59,8 @@ def parse():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-flush", action="store_true",
+                    help="do not flush L2 before each timed reuse / dense repetition")
     ap.add_argument("--shard", choices=["batch", "heads"], default="batch",
                     help="multi-GPU split: each rank its own batch element(s) (weak scaling) "
                          "or the workload's heads split over the ranks (strong scaling)")
@@ -171,14 +173,17 @@ def reference_arm(args, wl):
         v, done, el = oracle_reuse_sample(wl, per_step, Q1, K1, V1, sel, Rg, groups)
         vals.append(v)
         ms.append(el * 1e3 / done)
-    value = statistics.mean(vals)
+    value = statistics.median(vals)
     sample = (f"reuse-step sparse attention + residual, fp64, on whole {gs}-query groups of "
               f"head 0 over random ascending k={wl.k} subsets standing in for the cached "
-              f"selection, ~{per_step:.1f} s per step; TFLOP/s = executed flops / time")
+              f"selection, ~{per_step:.1f} s per step; TFLOP/s = executed flops / time; "
+              f"ms_per_step is extrapolated from the sample's time per group to all "
+              f"{wl.num_groups * wl.heads} groups of the workload")
     line = {
         "impl": "reference", "metric": METRIC, "value": value,
         "unit": "TFLOP/s (executed, reuse step)", "n_gpus": args.gpus, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": statistics.mean(ms) * wl.num_groups * wl.heads,
+        "warmup": args.warmup, "ms_per_step": statistics.median(ms) * wl.num_groups * wl.heads,
+        "ms_per_step_extrapolated": True,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic", "config": config_of(wl),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s (executed, reuse step)",
@@ -194,7 +199,9 @@ def config_of(wl):
             "n_kv": wl.n_kv, "head_dim": wl.head_dim, "group_size": wl.group_size, "k": wl.k,
             "kv_density": round(wl.k / wl.n_kv, 4), "input_dtype": wl.dtype,
             "step": "PDDP grouping + anchor step + one reuse step (drifted inputs)",
-            "l2": "inputs larger than L2: Q,K,V %.0f MB + R %.0f MB per step, no explicit flush"
+            "l2": "inputs larger than L2 (Q,K,V %.0f MB + R %.0f MB per step); the reuse and "
+                  "dense timings also flush L2 (write of a 512 MB buffer) before each "
+                  "repetition, medians reported"
                   % (3 * wl.batch * wl.heads * wl.n_kv * wl.head_dim * 2 / 1e6,
                      wl.batch * wl.heads * wl.n_q * wl.head_dim * 4 / 1e6)}
 
@@ -285,22 +292,37 @@ def main():
     total_ms = t_start.elapsed_time(t_end)
     group_ms = [e[0].elapsed_time(e[1]) for e in events]
     anchor_ms = [e[1].elapsed_time(e[2]) for e in events]
-    reuse_ms = [e[2].elapsed_time(e[3]) for e in events]
+    step_reuse_ms = [e[2].elapsed_time(e[3]) for e in events]
     if ws.status() != 0:
         raise RuntimeError(f"device status {tlsp.status_string(ws.status())} after timing")
 
-    # Dense pass alone (the comparison point of the reuse step).
-    dense_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    # The reuse step and the dense pass alone (the comparison point), each
+    # repetition after an L2 flush (a 512 MB write) so K/V come from HBM as
+    # they would on a fresh step.
+    flush_buf = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    def timed(fn, reps, flush):
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(reps)]
+        for _ in range(2):
+            fn()
+        for r in range(reps):
+            if flush:
+                flush_buf.fill_(r & 0xff)
+            ev[r][0].record()
+            fn()
+            ev[r][1].record()
+        torch.cuda.synchronize()
+        return [e[0].elapsed_time(e[1]) for e in ev]
+
+    flush = not args.no_flush
+    reuse_call = lambda: tlsp.reuse_attention(Qr, Kr, Vr, groups, gs, k, idx, R, ws, out=O)
+    launches_r0 = tlsp.launch_count()
+    reuse_ms = timed(reuse_call, args.steps, flush)
+    reuse_launches = (tlsp.launch_count() - launches_r0) // (args.steps + 2)
+    reuse_warm_ms = timed(reuse_call, args.steps, False)
     O_dense = torch.empty_like(Qa)
-    for _ in range(2):
-        tlsp.dense_attention(Qa, Ka, Va, ws, out=O_dense)
-    torch.cuda.synchronize()
-    for s in range(args.steps):
-        dense_ev[s][0].record()
-        tlsp.dense_attention(Qa, Ka, Va, ws, out=O_dense)
-        dense_ev[s][1].record()
-    torch.cuda.synchronize()
-    dense_ms = [e[0].elapsed_time(e[1]) for e in dense_ev]
+    dense_ms = timed(lambda: tlsp.dense_attention(Qa, Ka, Va, ws, out=O_dense), args.steps, flush)
+    del flush_buf
 
     # End to end through the C ABI with host buffers: pinned inputs in,
     # result out, copies inside the timed region (reuse steps).
@@ -322,10 +344,11 @@ def main():
     h2d = sum(t.numel() * t.element_size() for t in (Qr_h, Kr_h, Vr_h))
     d2h = O_h.numel() * O_h.element_size()
 
-    mx = max_over_ranks([total_ms, statistics.mean(reuse_ms), statistics.mean(anchor_ms),
-                         statistics.mean(group_ms), statistics.mean(dense_ms),
-                         statistics.mean(e2e_ms)])
-    total_ms, reuse_mean, anchor_mean, group_mean, dense_mean, e2e_mean = mx
+    med = statistics.median
+    mx = max_over_ranks([total_ms, med(reuse_ms), med(anchor_ms), med(group_ms), med(dense_ms),
+                         med(e2e_ms), med(reuse_warm_ms), med(step_reuse_ms)])
+    (total_ms, reuse_mean, anchor_mean, group_mean, dense_mean, e2e_mean, reuse_warm,
+     reuse_in_step) = mx
     flops = wl.reuse_flops()  # this rank's work
     # the whole job's work: world copies of the batch shard, or the full workload split by heads
     strong = args.shard == "heads"
@@ -350,7 +373,9 @@ def main():
         "config": dict(config_of(full_wl),
                        global_batch=full_wl.batch if strong else world * wl.batch,
                        parallelism=f"heads{world}" if strong else f"dp{world}"),
-        "reuse_ms": reuse_mean, "anchor_ms": anchor_mean, "group_queries_ms": group_mean,
+        "reuse_ms": reuse_mean, "reuse_ms_warm_l2": reuse_warm, "reuse_ms_in_step": reuse_in_step,
+        "reuse_launches": reuse_launches,
+        "anchor_ms": anchor_mean, "group_queries_ms": group_mean,
         "dense_pass_ms": dense_mean, "reuse_vs_dense_speedup": dense_mean / reuse_mean,
         "reuse_dense_equiv_tflops": job_dense / (reuse_mean * 1e-3) / 1e12,
         "dense_pass_tflops": wl.dense_flops() / (dense_mean * 1e-3) / 1e12,

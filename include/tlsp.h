@@ -48,7 +48,7 @@ typedef enum {
   TLSP_OK = 0,
   TLSP_ERR_INVALID_ARG = -1,   /* null pointer, bad shape, misaligned pointer, k > n_kv ... */
   TLSP_ERR_UNSUPPORTED = -2,   /* valid request this build has no kernel for */
-  TLSP_ERR_WORKSPACE = -3,     /* ws_bytes smaller than tlsp_workspace_bytes() */
+  TLSP_ERR_WORKSPACE = -3,     /* ws_bytes smaller than the call needs */
   TLSP_ERR_CUDA = -4,          /* a CUDA runtime call or launch failed */
   TLSP_ERR_TIMEOUT = -5,       /* device: a bounded wait ran out (kernel returned early) */
   TLSP_ERR_DEVICE_ASSERT = -6  /* device: an internal check failed (e.g. index out of range) */
@@ -76,8 +76,9 @@ int32_t tlsp_num_levels(int32_t n_q, int32_t group_size);
 
 /* Workspace bytes sufficient for every call below with these dims,
  * group_size and k (the maximum over calls). 0 on invalid arguments. The
- * anchor call's internal score buffer is included (B*H*G*n_kv floats) so a
- * NULL `scores` argument is always allowed. */
+ * anchor call scores and selects the (head, group) rows in batches of at
+ * most about 80 MB of fp32 scores; the workspace holds one batch (not the
+ * B*H*G*n_kv matrix), so a NULL `scores` argument is always allowed. */
 size_t tlsp_workspace_bytes(const tlsp_dims* dims, int32_t group_size, int32_t k);
 
 /* Tile-aligned query grouping by fast PDDP (review section 3: queries that
@@ -170,7 +171,14 @@ int tlsp_dense_attention_noalloc(const tlsp_dims* dims, const void* Q, const voi
  * the residual as an additive correction).
  *   Q, K, V   this step's inputs; groups, indices and R from the last anchor.
  *   O         out [B, H, n_q, d] in dims->dtype, token order:
- *             O_i = sparse attention of q_i over indices[g(i)] + R_i. */
+ *             O_i = sparse attention of q_i over indices[g(i)] + R_i.
+ *   ws        only its status word is used: 16-byte aligned and at least
+ *             256 bytes (a full tlsp_workspace_bytes() workspace also works).
+ * groups, indices and R are caller-kept state, checked on the device: a
+ * selection entry outside [0, n_kv), a group member outside [0, n_q), or a
+ * padding entry of the last group's ragged tail other than -1, records
+ * TLSP_ERR_DEVICE_ASSERT in the status word; the output of the tiles
+ * involved is then unspecified (the others are unaffected). */
 int tlsp_reuse_attention(const tlsp_dims* dims, const void* Q, const void* K, const void* V,
                          const int32_t* groups, int32_t group_size, int32_t k,
                          const int32_t* indices, const float* R, void* O, void* ws,

@@ -59,8 +59,12 @@ def test_group_counts(T):
 def test_workspace_bytes(T):
     d = T.Dims(1, 12, 32760, 32760, 128, T.TLSP_BF16)
     n = T.lib().tlsp_workspace_bytes(ctypes.byref(d), 128, 1664)
-    # must at least hold the internal fp32 score buffer [B, H, G, n_kv]
-    assert n >= 12 * 256 * 32760 * 4
+    # holds one batch of fp32 score rows (4 waves of 148 rows at n_kv = 32760),
+    # not the whole [B, H, G, n_kv] matrix
+    assert 592 * 32760 * 4 <= n < 12 * 256 * 32760 * 4
+    d4 = T.Dims(1, 40, 75600, 75600, 128, T.TLSP_BF16)
+    n4 = T.lib().tlsp_workspace_bytes(ctypes.byref(d4), 128, 7552)
+    assert 296 * 75600 * 4 <= n4 < 1 << 30
     assert T.lib().tlsp_workspace_bytes(ctypes.byref(d), 128, 32761) == 0   # k > n_kv
     bad = T.Dims(1, 12, 32760, 32760, 96, T.TLSP_BF16)
     assert T.lib().tlsp_workspace_bytes(ctypes.byref(bad), 128, 1) == 0     # head_dim
@@ -100,6 +104,11 @@ def test_validation_rejects_before_launch(T):
     assert L.tlsp_reuse_attention(ctypes.byref(d), p, p, p, p, 16, 32, p, None, p, p, big,
                                   None) == E_ARG
     assert L.tlsp_reuse_attention(ctypes.byref(d), p, p, odd, p, 16, 32, p, p, p, p, big,
+                                  None) == E_ARG
+    # the reuse step needs only the 256-byte status word
+    assert L.tlsp_reuse_attention(ctypes.byref(d), p, p, p, p, 16, 32, p, p, p, p, 255,
+                                  None) == E_WS
+    assert L.tlsp_reuse_attention(ctypes.byref(d), p, p, p, p, 16, 32, p, p, p, None, 256,
                                   None) == E_ARG
     assert L.tlsp_topk_from_scores(p, 4, 10, 11, p, None, 0, None) == E_ARG
     assert L.tlsp_split_from_projections(p, p, 8, 9, p, p, None, 0, None) == E_ARG

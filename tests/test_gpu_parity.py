@@ -55,9 +55,14 @@ def test_workload3_ar_chunk_sampled(T):
 
 @pytest.mark.slow
 def test_workload4_large_sampled(T):
+    # two heads: the 10-level PDDP tree (591 groups, nodes down to 2 slots)
+    # replayed against the oracle's fp64 projections, fed top-k on 64 rows per
+    # head, outputs on sampled groups including the ragged last one
     wl = workload(4)
-    assert_ok(run_and_compare(wl, sample_heads=[39], sample_groups=[5, 590], topk_rows=16,
-                              replay_own=False))
+    rep = run_and_compare(wl, sample_heads=[0, 39], sample_groups=[5, 300, 590], topk_rows=64,
+                          replay_own=True)
+    assert_ok(rep)
+    assert rep.errors["proj.rel_max"] <= 2e-3
 
 
 # ------------------------------------------------------------ edge cases
@@ -104,6 +109,24 @@ def test_topk_fed_ties_and_signed_zero(T):
             assert np.array_equal(idx[r], orc.topk(S[r].astype(np.float64), k)), (n_kv, k, r)
 
 
+def test_topk_fed_many_rows_and_shapes(T):
+    # more rows than the persistent grid (each CTA takes several rows), row
+    # lengths that are not a multiple of 4, attention-like heavy-tailed rows
+    # (the candidate-list path) and flat rows (the streaming fallback)
+    from oracle import oracle as orc
+    rng = np.random.default_rng(5)
+    for rows, n_kv, k in [(700, 4096, 205), (9, 4095, 200), (12, 32760, 1664), (4, 75600, 7552),
+                          (3, 130, 64)]:
+        S = rng.exponential(1.0, size=(rows, n_kv)).astype(np.float32) ** 3
+        S[0] = rng.standard_normal(n_kv).astype(np.float32)
+        S[1] = 1.0                       # every key tied
+        S[2, : n_kv // 2] = 0.5          # half the row tied, inside the selection's bin
+        idx = T.topk_from_scores(torch.from_numpy(S).cuda(), k).cpu().numpy()
+        check = range(rows) if rows <= 16 else list(range(8)) + list(range(rows - 8, rows))
+        for r in check:
+            assert np.array_equal(idx[r], orc.topk(S[r].astype(np.float64), k)), (n_kv, k, r)
+
+
 def test_split_fed_with_ties(T):
     from oracle import oracle as orc
     rng = np.random.default_rng(1)
@@ -147,6 +170,77 @@ def test_out_of_range_index_sets_device_status(T):
     ws.reset()
     torch.cuda.synchronize()
     assert ws.status() == T.TLSP_OK
+
+
+def _anchor_state(T, wl, gs, k):
+    from token_level_sparse_pddp_b200.synthetic import InputStream
+    it = iter(InputStream(wl))
+    _, _, Q, K, V = next(it)
+    _, _, Q1, K1, V1 = next(it)
+    Q, K, V, Q1, K1, V1 = (x.cuda() for x in (Q, K, V, Q1, K1, V1))
+    ws = T.Workspace(T.dims_of(Q, K), gs, k)
+    groups = T.group_queries(Q, gs, ws)
+    O, idx, R = T.anchor_attention(Q, K, V, groups, gs, k, ws)
+    torch.cuda.synchronize()
+    assert ws.status() == T.TLSP_OK
+    return ws, groups, idx, R, (Q1, K1, V1)
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64)])
+def test_negative_index_sets_device_status_and_spares_other_tiles(T, dtype, d):
+    # a negative selection entry is caller-kept state gone bad: the kernel
+    # records it before use, and every other group's output is unchanged
+    wl = small("neg-index", dtype=dtype, head_dim=d, grid=(2, 8, 10))   # 160 queries, ragged tail
+    gs, k = 16, 32
+    ws, groups, idx, R, (Q1, K1, V1) = _anchor_state(T, wl, gs, k)
+    clean = T.reuse_attention(Q1, K1, V1, groups, gs, k, idx, R, ws)
+    bad = idx.clone()
+    bad[0, 1, 3, 7] = -5
+    out = T.reuse_attention(Q1, K1, V1, groups, gs, k, bad, R, ws)
+    torch.cuda.synchronize()
+    assert ws.status() == T.TLSP_ERR_DEVICE_ASSERT
+    rows = groups[0, 1, 3 * gs:4 * gs].long()
+    keep = torch.ones(out.shape[2], dtype=torch.bool, device=out.device)
+    keep[rows[rows >= 0]] = False
+    assert torch.equal(out[0, 0], clean[0, 0])
+    assert torch.equal(out[0, 1][keep], clean[0, 1][keep])
+    ws.reset()
+    torch.cuda.synchronize()
+    assert ws.status() == T.TLSP_OK
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64)])
+def test_bad_group_entries_set_device_status(T, dtype, d):
+    # -1 is padding only in the ragged tail of the last group; a -1 among a
+    # full group's members, or a token id in the tail, is recorded
+    wl = small("bad-group", dtype=dtype, head_dim=d, grid=(2, 8, 10))   # G = 10, last holds 16
+    gs, k = 16, 32
+    wl2 = small("bad-group-ragged", dtype=dtype, head_dim=d, grid=(3, 5, 10))  # 150 = 9*16 + 6
+    for w, plant in ((wl, (0, 1, 5 * 16 + 5, -1)), (wl2, (0, 0, 9 * 16 + 10, 3))):
+        ws, groups, idx, R, (Q1, K1, V1) = _anchor_state(T, w, gs, k)
+        T.reuse_attention(Q1, K1, V1, groups, gs, k, idx, R, ws)
+        torch.cuda.synchronize()
+        assert ws.status() == T.TLSP_OK
+        b, h, pos, val = plant
+        bad = groups.clone()
+        bad[b, h, pos] = val
+        T.reuse_attention(Q1, K1, V1, bad, gs, k, idx, R, ws)
+        torch.cuda.synchronize()
+        assert ws.status() == T.TLSP_ERR_DEVICE_ASSERT, (w.name, plant)
+
+
+@pytest.mark.parametrize("dtype,d", [("bf16", 128), ("f32", 64)])
+def test_reuse_needs_only_the_status_word(T, dtype, d):
+    wl = small("reuse-ws", dtype=dtype, head_dim=d)
+    gs, k = 16, 32
+    ws, groups, idx, R, (Q1, K1, V1) = _anchor_state(T, wl, gs, k)
+    full = T.reuse_attention(Q1, K1, V1, groups, gs, k, idx, R, ws)
+    tiny = T.Workspace.status_only()
+    assert tiny.nbytes == 256
+    out = T.reuse_attention(Q1, K1, V1, groups, gs, k, idx, R, tiny)
+    torch.cuda.synchronize()
+    assert tiny.status() == T.TLSP_OK
+    assert torch.equal(out, full)
 
 
 def test_bounded_wait_times_out_and_context_survives(T):

@@ -4,8 +4,9 @@ Some callers cannot allocate device memory or hand over a workspace (code
 running while a CUDA graph is captured, or under a framework whose memory
 pool owns all allocations). tlsp_dense_attention_noalloc serves them from a
 fixed scratch array inside the library. This file checks, through the C ABI,
-that it returns what tlsp_dense_attention returns, on two calls in a row, and
-that requests larger than its fixed scratch are refused. It is named so that
+that it returns what tlsp_dense_attention returns, on two calls in a row,
+that sampled rows agree with the fp64 oracle's dense attention, and that
+requests larger than its fixed scratch are refused. It is named so that
 pytest collects it last.
 """
 import ctypes
@@ -46,6 +47,16 @@ def test_noalloc_matches_workspace_entry_point(T, dtype, B, H, n_q, n_kv, d):
         diff = (out.float() - ref.float()).abs()
         assert diff.max().item() <= max_tol and diff.mean().item() <= mean_tol
     assert ws.status() == T.TLSP_OK
+    # both entry points run the same dense kernel, so also hold a few rows of
+    # each head against the fp64 oracle's dense attention on the same inputs
+    from oracle import oracle as orc
+    rows = [0, n_q // 2, n_q - 1]
+    for b in range(B):
+        for h in range(H):
+            Xq, Xk, Xv = (X[b, h].double().cpu().numpy() for X in (Q, K, V))
+            O_ref, _ = orc.dense(Xq[rows], Xk, Xv)
+            d_or = abs(out[b, h, rows].double().cpu().numpy() - O_ref)
+            assert d_or.max() <= max_tol and d_or.mean() <= mean_tol, (b, h, d_or.max())
 
 
 def test_noalloc_refuses_sizes_beyond_its_scratch(T):

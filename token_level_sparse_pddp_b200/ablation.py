@@ -18,6 +18,13 @@ step's selection and sparse work:
                 the reuse steps), block-granular selection, no residual;
   exact_token   as exact_block with token-level selection;
   pddp_token    as exact_token with PDDP query groups;
+  recompute_token
+                as pddp_token, but the exact token selection is made again on
+                every step from that step's own exact scores (the groups are
+                still the anchor's): set against pddp_token on the reuse steps
+                it isolates what reusing an anchor's selection costs in error
+                (the review's case for reuse is the temporal stability of the
+                selections) and what recomputing it costs in time;
   mc_sparse     as pddp_token with the dense-sparse residual R added back.
 
 On an anchor step every variant except bsa runs the dense pass anyway (exact
@@ -36,7 +43,7 @@ import torch
 from . import tlsp
 from .synthetic import InputStream, workload
 
-VARIANTS = ("bsa", "exact_block", "exact_token", "pddp_token", "mc_sparse")
+VARIANTS = ("bsa", "exact_block", "exact_token", "pddp_token", "recompute_token", "mc_sparse")
 
 
 def rel_l2(O: torch.Tensor, O_ref: torch.Tensor) -> float:
@@ -52,7 +59,10 @@ def rel_l2_head_mean(O: torch.Tensor, O_ref: torch.Tensor) -> float:
                   torch.linalg.vector_norm(r, dim=2)).mean())
 
 
-def run(wl, block: int, steps: int = 0) -> List[Dict]:
+def run(wl, block: int, steps: int = 0, record: Dict = None) -> List[Dict]:
+    """The ladder on the workload's schedule. With `record` (a dict), the
+    recompute_token variant's groups, selection and exact scores of every
+    reuse step are kept in it under the step number."""
     if wl.n_kv % block or wl.k % block:
         raise ValueError(f"block {block} must divide n_kv={wl.n_kv} and k={wl.k}")
     dev = torch.device("cuda")
@@ -84,6 +94,15 @@ def run(wl, block: int, steps: int = 0) -> List[Dict]:
                     idx = tlsp.pooled_block_select(Q, K, raster, gs, k, block, ws)
                     return tlsp.reuse_attention(Q, K, V, raster, gs, k, idx, R0, ws)
                 O, ms = timed(step)
+            elif v == "recompute_token" and kind != "A":
+                def step():
+                    _, idx, _, S = tlsp.anchor_attention(Q, K, V, st["groups"], gs, k, ws,
+                                                         return_scores=True)
+                    return tlsp.reuse_attention(Q, K, V, st["groups"], gs, k, idx, R0, ws), idx, S
+                (O, idx, S), ms = timed(step)
+                if record is not None:
+                    record[s] = dict(groups=st["groups"], idx=idx, S=S)
+                del S
             elif kind == "A":
                 def step():
                     groups = raster if v in ("exact_block", "exact_token") else \
@@ -115,12 +134,14 @@ DECOMPOSITION = (
 )
 
 
-def decompose(wl, block: int) -> List[Dict]:
+def decompose(wl, block: int, return_selections: bool = False):
     """The review's three sparse-attention errors (structural binding, selection,
     discarded tail) taken apart on the first step of a workload: each row adds one
     source of error to the one before and reports the rel-L2 of the sparse output
     (no residual) against dense attention. Per-query selection is the library's
-    grouping with group size 1."""
+    grouping with group size 1. With return_selections, also returns the
+    inputs (Q, K, V on the host) and each rung's (groups, group size,
+    selection) on the host, so the same selections can be evaluated elsewhere."""
     if wl.n_kv % block or wl.k % block:
         raise ValueError(f"block {block} must divide n_kv={wl.n_kv} and k={wl.k}")
     dev = torch.device("cuda")
@@ -133,7 +154,11 @@ def decompose(wl, block: int) -> List[Dict]:
     R0 = torch.zeros(Q.shape, dtype=torch.float32, device=dev)
     out = []
 
+    sels = []
+
     def sparse(groups, g, idx, w):
+        if return_selections:
+            sels.append((groups.cpu().numpy(), g, idx.cpu().numpy()))
         return tlsp.reuse_attention(Q, K, V, groups, g, k, idx, R0, w)
 
     single = tlsp.group_raster(Q, 1)
@@ -151,9 +176,12 @@ def decompose(wl, block: int) -> List[Dict]:
     torch.cuda.synchronize()
     if ws.status() != 0:
         raise RuntimeError(f"device status {tlsp.status_string(ws.status())}")
-    return [dict(component=c, what=w, rel_l2=rel_l2(O, O_dense),
+    rows = [dict(component=c, what=w, rel_l2=rel_l2(O, O_dense),
                  rel_l2_head_mean=rel_l2_head_mean(O, O_dense))
             for (c, w), O in zip(DECOMPOSITION, out)]
+    if return_selections:
+        return rows, (Q.cpu(), K.cpu(), V.cpu()), sels
+    return rows
 
 
 def main():

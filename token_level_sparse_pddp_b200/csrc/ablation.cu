@@ -74,8 +74,7 @@ int launch_block_topk(const float* in, int64_t rows, int n_in, int n_blocks, int
   if (rows == 0) return TLSP_OK;
   const size_t smem = block_topk_smem(n_blocks, kb);
   if (smem > (size_t)kBlockSmemMax || rows > 0x7fffffffLL) return TLSP_ERR_UNSUPPORTED;
-  cudaFuncSetAttribute(block_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       kBlockSmemMax);
+  TLSP_TRY(ensure_smem_limit((const void*)block_topk_kernel, kBlockSmemMax));
   block_topk_kernel<<<(unsigned)rows, kSelectThreads, smem, st>>>(in, n_in, n_blocks, sum_width,
                                                                   kb, b_expand, indices, block_out);
   return check_launch();

@@ -1,6 +1,10 @@
 // C ABI of libtlsp (declared in include/tlsp.h): argument validation,
 // workspace layout and dispatch to the kernels.
+#include <algorithm>
 #include <cstdio>
+#include <mutex>
+#include <tuple>
+#include <vector>
 
 #include "kernels.h"
 
@@ -10,13 +14,70 @@ std::atomic<int64_t> g_launch_count{0};
 static thread_local int t_last_cuda_error = 0;
 void set_last_cuda_error(cudaError_t e) { t_last_cuda_error = (int)e; }
 
+// ----------------------------------------------------------------- per-device launch facts
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+std::mutex g_attr_mu;
+std::vector<std::tuple<const void*, int, int>> g_attr_done;  // (kernel, device, bytes)
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+}  // namespace
+
+int device_sm_count() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  int n = g_sm_count[dev].load(std::memory_order_relaxed);
+  if (n <= 0) {
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    g_sm_count[dev].store(n, std::memory_order_relaxed);
+  }
+  return n;
+}
+
+int ensure_smem_limit(const void* fn, int bytes) {
+  const int dev = current_device();
+  std::lock_guard<std::mutex> lock(g_attr_mu);
+  for (const auto& t : g_attr_done)
+    if (std::get<0>(t) == fn && std::get<1>(t) == dev && std::get<2>(t) >= bytes) return TLSP_OK;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) {
+    set_last_cuda_error(e);
+    return TLSP_ERR_CUDA;
+  }
+  g_attr_done.emplace_back(fn, dev, bytes);
+  return TLSP_OK;
+}
+
 // ----------------------------------------------------------------- workspace
 
 constexpr size_t kAlign = 256;
 constexpr size_t kStatusBytes = 256;  // status word at 0, debug flag at 64
 constexpr int64_t kPddpPartialSlots = 640;
+// The anchor step scores and selects (head, group) rows in batches of about
+// this many score bytes: a batch's scores are still in L2 when the selection
+// reads them, and the workspace holds one batch, not every row.
+constexpr size_t kScoreBatchBytes = size_t(80) << 20;
+constexpr int64_t kBatchRowQuantum = 148;  // whole waves of the score kernel on a B200
 
 static size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Rows (head, group) per score batch: every row when they fit, else as many
+// whole waves of kBatchRowQuantum rows as fit in kScoreBatchBytes (at least
+// one row; at most 65535, the score launch's limit).
+static int64_t score_batch_rows(const tlsp_dims& d, int gs) {
+  const int64_t total = (int64_t)d.batch * d.heads * ((d.n_q + gs - 1) / gs);
+  int64_t per = (int64_t)(kScoreBatchBytes / (sizeof(float) * (size_t)d.n_kv));
+  if (per >= kBatchRowQuantum) per = per / kBatchRowQuantum * kBatchRowQuantum;
+  per = std::max<int64_t>(1, std::min<int64_t>(per, 65535));
+  return std::min(total, per);
+}
 
 struct Layout {
   size_t lse, scores, perm, tmp, seg_key, node_mu, node_v, partials, total;
@@ -33,7 +94,7 @@ static Layout layout_of(const tlsp_dims& d, int gs) {
     return at;
   };
   L.lse = take(sizeof(float) * BH * d.n_q);
-  L.scores = take(sizeof(float) * BH * G * d.n_kv);
+  L.scores = take(sizeof(float) * (size_t)score_batch_rows(d, gs) * d.n_kv);
   L.perm = take(sizeof(int32_t) * BH * d.n_q);
   L.tmp = take(sizeof(int32_t) * BH * d.n_q);
   L.seg_key = take(sizeof(uint32_t) * BH * d.n_q);
@@ -188,10 +249,15 @@ int tlsp_anchor_attention(const tlsp_dims* dims, const void* Q, const void* K, c
   cudaStream_t st = (cudaStream_t)stream;
   const AttnArgs a = attn_args(dims, Q, K, V, group_size, k, ws);
   float* lse = at<float>(ws, L.lse);
-  float* S = scores ? scores : at<float>(ws, L.scores);
   TLSP_TRY(dense_pass(a, O, lse, st));
-  TLSP_TRY(scores_pass(a, groups, lse, S, st));
-  TLSP_TRY(launch_topk(S, a.BH * a.G, a.n_kv, k, indices, a.status, st));
+  // exact scores and the top-k selection, batch by batch of (head, group) rows
+  const int64_t total = a.BH * a.G, per = score_batch_rows(*dims, group_size);
+  for (int64_t r0 = 0; r0 < total; r0 += per) {
+    const int64_t rows = std::min(per, total - r0);
+    float* S = scores ? scores + r0 * a.n_kv : at<float>(ws, L.scores);
+    TLSP_TRY(scores_pass(a, groups, lse, S, r0, rows, st));
+    TLSP_TRY(launch_topk(S, rows, a.n_kv, k, indices + r0 * k, a.status, st));
+  }
   return sparse_pass(a, groups, indices, O, R, nullptr, nullptr, st);
 }
 
@@ -217,7 +283,9 @@ int tlsp_reuse_attention(const tlsp_dims* dims, const void* Q, const void* K, co
   if (!Q || !K || !V || !groups || !O || !indices || !R) return TLSP_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(R))
     return TLSP_ERR_INVALID_ARG;
-  TLSP_TRY(check_ws(dims, group_size, ws, ws_bytes));
+  // the reuse step's only scratch is the status word
+  if (!ws || !aligned16(ws)) return TLSP_ERR_INVALID_ARG;
+  if (ws_bytes < kStatusBytes) return TLSP_ERR_WORKSPACE;
   const AttnArgs a = attn_args(dims, Q, K, V, group_size, k, ws);
   return sparse_pass(a, groups, indices, nullptr, nullptr, R, O, (cudaStream_t)stream);
 }

@@ -97,11 +97,12 @@ template <class T, int D>
 __global__ void __launch_bounds__(128)
 scores_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const float* __restrict__ LSE,
                    const int32_t* __restrict__ groups, int n_q, int n_kv, int gs, int G,
-                   float scale, float* __restrict__ S, int* status) {
+                   int64_t row0, float scale, float* __restrict__ S, int* status) {
   __shared__ __align__(16) float q_s[32][D];
   __shared__ float lse_s[32];
-  const int g = blockIdx.y;
-  const int64_t bh = blockIdx.z;
+  const int64_t grow = row0 + blockIdx.y;  // (head, group) row; S holds this launch's rows
+  const int g = (int)(grow % G);
+  const int64_t bh = grow / G;
   const int j = blockIdx.x * 128 + threadIdx.x;
   const int32_t* grp = groups + (bh * G + g) * (int64_t)gs;
   const T* kj = K + (bh * n_kv + min(j, n_kv - 1)) * D;
@@ -127,7 +128,7 @@ scores_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const float
       }
     }
   }
-  if (j < n_kv) S[(bh * G + g) * (int64_t)n_kv + j] = acc;
+  if (j < n_kv) S[(int64_t)blockIdx.y * n_kv + j] = acc;
 }
 
 // Gathered sparse attention over indices[bh, g, 0..k) with the residual
@@ -147,11 +148,14 @@ sparse_simt_kernel(const T* __restrict__ Q, const T* __restrict__ K, const T* __
   const int64_t bh = blockIdx.z;
   if (r >= gs) return;
   const int tok = groups[(bh * G + g) * (int64_t)gs + r];
-  if (tok < 0) return;  // padding row of the ragged last group
-  if (tok >= n_q) {
+  // members of a group are token ids in [0, n_q); only the ragged tail of
+  // the last group holds padding, and padding is -1
+  const int members = g == G - 1 ? n_q - (G - 1) * gs : gs;
+  if (r < members ? (tok < 0 || tok >= n_q) : tok != -1) {
     if (lane == 0) record_status(status, TLSP_ERR_DEVICE_ASSERT);
     return;
   }
+  if (tok < 0) return;  // padding row of the ragged last group
   const T* q = Q + (bh * n_q + tok) * D;
   for (int c = lane; c < D; c += 32) q_s[warp][c] = to_f32(q[c]);
   __syncwarp();
@@ -193,10 +197,13 @@ static int dense_t(const AttnArgs& a, void* O, float* LSE, cudaStream_t st) {
 
 template <class T, int D>
 static int scores_t(const AttnArgs& a, const int32_t* groups, const float* LSE, float* S,
-                    cudaStream_t st) {
-  dim3 grid((unsigned)ceil_div(a.n_kv, 128), (unsigned)a.G, (unsigned)a.BH);
+                    int64_t row0, int64_t rows, cudaStream_t st) {
+  if (rows <= 0) return TLSP_OK;
+  if (rows > 65535) return TLSP_ERR_UNSUPPORTED;
+  dim3 grid((unsigned)ceil_div(a.n_kv, 128), (unsigned)rows);
   scores_simt_kernel<T, D><<<grid, 128, 0, st>>>((const T*)a.Q, (const T*)a.K, LSE, groups, a.n_q,
-                                                 a.n_kv, a.gs, a.G, rsqrtf((float)D), S, a.status);
+                                                 a.n_kv, a.gs, a.G, row0, rsqrtf((float)D), S,
+                                                 a.status);
   return check_launch();
 }
 
@@ -225,8 +232,8 @@ int simt_dense(const AttnArgs& a, void* O, float* LSE, cudaStream_t st) {
   return TLSP_DISPATCH(dense_t, a, O, LSE, st);
 }
 int simt_scores(const AttnArgs& a, const int32_t* groups, const float* LSE, float* S,
-                cudaStream_t st) {
-  return TLSP_DISPATCH(scores_t, a, groups, LSE, S, st);
+                int64_t row0, int64_t rows, cudaStream_t st) {
+  return TLSP_DISPATCH(scores_t, a, groups, LSE, S, row0, rows, st);
 }
 int simt_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices,
                 const void* O_full, float* R_out, const float* R_in, void* O_out,

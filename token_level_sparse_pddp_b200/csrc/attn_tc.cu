@@ -16,9 +16,8 @@
 //              shared memory and gather its Q rows, then warps 4-7 gather the
 //              K rows and warps 8-11 the V rows of each chunk of 128 selected
 //              keys, with 16-byte cp.async (eight issuing warps: the gather
-//              rate grows with the warps that issue, not only with the bytes
-//              in flight), into 128-byte swizzled shared memory (the tcgen05
-//              canonical layout);
+//              rate grows with the warps that issue), into 128-byte swizzled
+//              shared memory (the tcgen05 canonical layout);
 //   warp 12    allocates TMEM; lane 0 issues the tcgen05.mma instructions.
 // Per chunk j: S_j = Q K_j^T (M=N=K=128, fp32 in TMEM), online softmax with
 // exp2 on the SFU (S read from TMEM 64 columns at a time, the second half
@@ -35,6 +34,10 @@
 // alike, which cancels exactly in O / l.
 // Every wait is bounded (1 s); on expiry the kernel records
 // TLSP_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
+// Index checks: a selection entry outside [0, n_kv), a group entry outside
+// [0, n_q) before the ragged tail of the last group, or one other than -1
+// inside it, is recorded as TLSP_ERR_DEVICE_ASSERT (that key is read as a
+// zero row, that query row is skipped); such a tile's output is unspecified.
 #include "kernels.h"
 #include "tc_ptx.cuh"
 
@@ -91,6 +94,26 @@ __device__ __forceinline__ void prefetch_l2(const void* ptr) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
 }
 
+// Members of group g: every group holds gs tokens except the last, which
+// holds n_q - (G-1)*gs followed by -1 padding.
+__device__ __forceinline__ int members_of(const AttnParams& p, int g) {
+  return g == p.G - 1 ? p.n_q - (p.G - 1) * p.gs : p.gs;
+}
+
+// Token of row gr of a group, or -1 for a padding row. A member entry
+// outside [0, n_q), or a padding entry other than -1, is recorded.
+__device__ __forceinline__ int group_token(const int32_t* grp, int gr, int members,
+                                           const AttnParams& p) {
+  if (gr >= p.gs) return -1;
+  const int tok = __ldg(grp + gr);
+  const bool ok = gr < members ? (tok >= 0 && tok < p.n_q) : tok == -1;
+  if (!ok) {
+    record_status(p.status, TLSP_ERR_DEVICE_ASSERT);
+    return -1;
+  }
+  return tok;
+}
+
 // Sparse tiles: pulls into L2 what the prologue and epilogue of tile nb read
 // from HBM: its selection, its query rows and the rows its epilogue reads
 // (R for the reuse step, O_full for the anchor step). Called by the 128
@@ -133,7 +156,8 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
 // Gathers a [128 x 128] bf16 tile whose row r is global row rows(r) (or
 // zeros for rows(r) < 0) with NT threads; thread pt copies 16-byte chunk
 // c = pt % 16 of rows it * (NT / 16) + pt / 16, so a warp instruction moves
-// two whole 256-byte rows.
+// two whole 256-byte rows (a thread per 16 bytes of a row: measured twice as
+// fast as a thread per row, whose instructions touch 32 rows each).
 template <int NT>
 __device__ __forceinline__ void gather_rows(uint32_t dst, const __nv_bfloat16* src,
                                             const int (&rows)[2048 / NT], int pt) {
@@ -147,19 +171,31 @@ __device__ __forceinline__ void gather_rows(uint32_t dst, const __nv_bfloat16* s
   }
 }
 
-// Global rows of chunk j of the selection for a producer thread of NT
-// (sel points at the selection in shared or global memory).
+// Global rows of chunk j of the selection for a producer thread of NT: read
+// from shared memory at sel_smem when the selection was staged there (an
+// explicit shared load), else from global memory at sel. Positions past k
+// are padding (-1); a selected entry outside [0, n_kv) is recorded and read
+// as a zero row.
 template <int NT>
-__device__ __forceinline__ void chunk_rows(const int32_t* sel, int j, int k, int n_kv, int pt,
+__device__ __forceinline__ void chunk_rows(const int32_t* sel, uint32_t sel_smem, bool staged,
+                                           int j, int k, int n_kv, int pt,
                                            int (&rows)[2048 / NT], int* status) {
 #pragma unroll
   for (int it = 0; it < 2048 / NT; ++it) {
     const int q = j * kTile + it * (NT / 16) + (pt >> 4);
-    rows[it] = q < k ? sel[q] : -1;
+    int v = -1;
+    if (q < k) {
+      if (staged)
+        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(sel_smem + 4u * (uint32_t)q));
+      else
+        v = __ldg(sel + q);
+    }
+    rows[it] = v;
   }
 #pragma unroll
   for (int it = 0; it < 2048 / NT; ++it) {
-    if (rows[it] >= n_kv) {
+    const int q = j * kTile + it * (NT / 16) + (pt >> 4);
+    if (q < k && (unsigned)rows[it] >= (unsigned)n_kv) {
       record_status(status, TLSP_ERR_DEVICE_ASSERT);
       rows[it] = -1;
     }
@@ -193,6 +229,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int rem = blockIdx.x % tiles_per_head;
   const int g = rem / p.tiles_per_group;
   const int t = rem % p.tiles_per_group;
+  const int members = members_of(p, g);
   const int32_t* grp = p.groups + (bh * p.G + g) * (int64_t)p.gs;
   const int32_t* sel = p.indices + (bh * p.G + g) * (int64_t)p.k;
   const int n_keys = p.k;
@@ -240,24 +277,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                      : "memory");
       asm volatile("cp.async.commit_group;" ::: "memory");
     }
-    const int32_t* selp = idx_smem ? reinterpret_cast<const int32_t*>(smem + kSmIdx) : sel;
     {
-      // all 128 gather Q; then warps 4-5 stream K chunks and warps 6-7 V chunks
+      // all 256 gather Q; then warps 4-7 stream K chunks and warps 8-11 V chunks
       const __nv_bfloat16* Qbh = p.Q + bh * (int64_t)p.n_q * kD;
       {
         int rows[8];
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int gr = t * kTile + it * 16 + (pt >> 4);
-          rows[it] = gr < p.gs ? __ldg(grp + gr) : -1;
-        }
-#pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          if (rows[it] >= p.n_q) {
-            record_status(p.status, TLSP_ERR_DEVICE_ASSERT);
-            rows[it] = -1;
-          }
-        }
+        for (int it = 0; it < 8; ++it)
+          rows[it] = group_token(grp, t * kTile + it * 16 + (pt >> 4), members, p);
         gather_rows<256>(base + kSmQ, Qbh, rows, pt);
         ptx::cp_async_arrive_noinc(&bars.q_full);
       }
@@ -274,7 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint64_t* full = is_k ? bars.k_full : bars.v_full;
       uint64_t* empty = is_k ? bars.k_empty : bars.v_empty;
       int rows[16];
-      chunk_rows<128>(selp, 0, p.k, p.n_kv, qt, rows, p.status);
+      chunk_rows<128>(sel, base + kSmIdx, idx_smem, 0, p.k, p.n_kv, qt, rows, p.status);
       for (int j = 0; j < n_chunks; ++j) {
         const int s = j % nslots, u = j / nslots;
         if (u > 0 && !ptx::mbar_wait(&empty[s], (u - 1) & 1, abort_flag, kWaitNs)) {
@@ -283,7 +310,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         gather_rows<128>(slot0 + s * kTileBytes, src, rows, qt);
         ptx::cp_async_arrive_noinc(&full[s]);
-        if (j + 1 < n_chunks) chunk_rows<128>(selp, j + 1, p.k, p.n_kv, qt, rows, p.status);
+        if (j + 1 < n_chunks)
+          chunk_rows<128>(sel, base + kSmIdx, idx_smem, j + 1, p.k, p.n_kv, qt, rows, p.status);
       }
       }
       if (pt < 128 && p.wave > 0 && (int64_t)blockIdx.x + p.wave < (int64_t)gridDim.x)
@@ -342,9 +370,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ softmax
     const int r = tid;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    const int gr = t * kTile + r;
-    int tok = gr < p.gs ? grp[gr] : -1;
-    if (tok >= p.n_q) tok = -1;
+    const int tok = group_token(grp, t * kTile + r, members, p);
     if (tok >= 0) {  // the row the epilogue reads, towards L2 while the tile computes
       const int64_t row = (bh * p.n_q + tok) * kD;
       if (kMode == kReuse) {
@@ -499,7 +525,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::tmem_ld32(tl + kTmO + q * 32, o);
         if (has_row && q < 3) load_block(q + 1, (q + 1) & 1);
         ptx::tmem_ld_wait(o);
-        if (tok < 0) continue;
+        if (!has_row) continue;  // (no warp-collective instruction follows in this iteration)
         const int c0 = q * 32;
         if (kMode == kAnchor) {
           float4* dst = reinterpret_cast<float4*>(p.R_out + row + c0);
@@ -549,10 +575,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int kMode>
-void launch(const AttnParams& p, int64_t tiles, cudaStream_t st) {
-  cudaFuncSetAttribute(attn_tc_kernel<kMode>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)kSmemBytes);
+int launch(const AttnParams& p, int64_t tiles, cudaStream_t st) {
+  TLSP_TRY(ensure_smem_limit((const void*)attn_tc_kernel<kMode>, (int)kSmemBytes));
   attn_tc_kernel<kMode><<<(unsigned)tiles, kThreads, kSmemBytes, st>>>(p);
+  return check_launch();
 }
 
 AttnParams base_params(const AttnArgs& a) {
@@ -568,10 +594,7 @@ AttnParams base_params(const AttnArgs& a) {
   p.tiles_per_group = (a.gs + kTile - 1) / kTile;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
   p.status = a.status;
-  int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  p.wave = sms;
+  p.wave = device_sm_count();
   return p;
 }
 
@@ -591,11 +614,8 @@ int tc_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices,
   p.O_out = (__nv_bfloat16*)O_out;
   const int64_t tiles = a.BH * a.G * p.tiles_per_group;
   if (tiles > 0x7fffffffLL) return TLSP_ERR_UNSUPPORTED;
-  if (R_out)
-    launch<kAnchor>(p, tiles, st);
-  else
-    launch<kReuse>(p, tiles, st);
-  return check_launch();
+  if (R_out) return launch<kAnchor>(p, tiles, st);
+  return launch<kReuse>(p, tiles, st);
 }
 
 }  // namespace tlsp

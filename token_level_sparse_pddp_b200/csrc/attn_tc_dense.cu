@@ -387,8 +387,7 @@ int tc_dense(const AttnArgs& a, void* O, float* lse, cudaStream_t st) {
   p.status = a.status;
   const int64_t tiles = a.BH * p.q_tiles;
   if (tiles > 0x7fffffffLL) return TLSP_ERR_UNSUPPORTED;
-  cudaFuncSetAttribute(attn_dense_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)kSmemBytes);
+  TLSP_TRY(ensure_smem_limit((const void*)attn_dense_tc_kernel, (int)kSmemBytes));
   attn_dense_tc_kernel<<<(unsigned)tiles, kThreads, kSmemBytes, st>>>(p);
   return check_launch();
 }

@@ -6,7 +6,9 @@
 // S_g[j] = sum_{i in g} exp(q_i . k_j / sqrt(d) - LSE_i), with LSE_i the log
 // partition of query i from the dense pass.
 //
-// One CTA per (head, group) for groups of at most 128 queries. The CTA keeps
+// One CTA per (head, group) row for groups of at most 128 queries; a launch
+// covers a contiguous range of rows (the anchor step goes through them in
+// batches whose scores stay in L2 for the selection that follows). The CTA keeps
 // the group's Q rows in shared memory and streams all keys in chunks of 128
 // with TMA box loads (four slots). The product is taken transposed,
 // S^T = K_chunk Q_g^T (M = 128 keys on TMEM lanes, N = 128 queries on TMEM
@@ -57,7 +59,8 @@ struct ScoreParams {
   const __nv_bfloat16* __restrict__ Q;
   const int32_t* __restrict__ groups;
   const float* __restrict__ lse;
-  float* __restrict__ S;
+  float* __restrict__ S;  // rows row0 .. row0 + gridDim.x - 1, from S[0]
+  int64_t row0;           // first (head, group) row of this launch
   int n_q, n_kv, gs, G;
   float scale_log2;
   int* status;
@@ -84,8 +87,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = &bars.abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t bh = blockIdx.x / p.G;
-  const int g = blockIdx.x % p.G;
+  const int64_t grow = p.row0 + blockIdx.x;
+  const int64_t bh = grow / p.G;
+  const int g = (int)(grow % p.G);
   const int32_t* grp = p.groups + (bh * p.G + g) * (int64_t)p.gs;
   const int n_chunks = (p.n_kv + kTile - 1) / kTile;
 
@@ -203,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     asm volatile("bar.sync 2, 256;" ::: "memory");
     const float4* l4 = reinterpret_cast<const float4*>(lse2_s);
     const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16) + h * kTile;
-    float* out = p.S + (bh * p.G + g) * (int64_t)p.n_kv;
+    float* out = p.S + (int64_t)blockIdx.x * p.n_kv;
     for (int j = h; j < n_chunks; j += 2) {
       if (!ptx::mbar_wait(&bars.s_full[h], (j >> 1) & 1, abort_flag, kWaitNs)) {
         fail(bars, p.status);
@@ -255,8 +259,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 bool tc_scores_supported(const AttnArgs& a) { return a.bf16 && a.d == kD && a.gs <= kTile; }
 
-int tc_scores(const AttnArgs& a, const int32_t* groups, const float* lse, float* S,
-              cudaStream_t st) {
+int tc_scores(const AttnArgs& a, const int32_t* groups, const float* lse, float* S, int64_t row0,
+              int64_t rows, cudaStream_t st) {
   ScoreParams p{};
   if ((uint64_t)a.BH * (uint64_t)a.n_kv >= 0x7fffffffull) return TLSP_ERR_UNSUPPORTED;
   TLSP_TRY(make_tmap_bf16_rows(&p.tmK, a.K, (uint64_t)a.BH * a.n_kv, kD, 64, kTile));
@@ -264,17 +268,17 @@ int tc_scores(const AttnArgs& a, const int32_t* groups, const float* lse, float*
   p.groups = groups;
   p.lse = lse;
   p.S = S;
+  p.row0 = row0;
   p.n_q = a.n_q;
   p.n_kv = a.n_kv;
   p.gs = a.gs;
   p.G = a.G;
   p.scale_log2 = 1.4426950408889634f / sqrtf((float)kD);
   p.status = a.status;
-  const int64_t ctas = a.BH * a.G;
-  if (ctas > 0x7fffffffLL) return TLSP_ERR_UNSUPPORTED;
-  cudaFuncSetAttribute(scores_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)kSmemBytes);
-  scores_tc_kernel<<<(unsigned)ctas, kThreads, kSmemBytes, st>>>(p);
+  if (rows <= 0) return TLSP_OK;
+  if (rows > 0x7fffffffLL) return TLSP_ERR_UNSUPPORTED;
+  TLSP_TRY(ensure_smem_limit((const void*)scores_tc_kernel, (int)kSmemBytes));
+  scores_tc_kernel<<<(unsigned)rows, kThreads, kSmemBytes, st>>>(p);
   return check_launch();
 }
 

@@ -35,6 +35,12 @@ inline int check_launch() {
 
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// Multiprocessor count of the current device, looked up once per device.
+int device_sm_count();
+// Raises kernel `fn`'s dynamic shared memory limit to `bytes` on the current
+// device; the attribute call is made once per (kernel, device, size).
+int ensure_smem_limit(const void* fn, int bytes);
+
 // ----------------------------------------------------------------- device side
 
 // Device status word: the first error wins, later ones are dropped.

@@ -47,8 +47,9 @@ int simt_dense(const AttnArgs& a, void* O, float* LSE, cudaStream_t st);
 int launch_pooled_select(const AttnArgs& a, const int32_t* groups, int block, int32_t* indices,
                          float* block_scores, float* scratch, cudaStream_t st);
 size_t pooled_scratch_floats(const AttnArgs& a, int block);
+// scores of the (head, group) rows row0 .. row0 + rows - 1 into S[0 .. rows * n_kv)
 int simt_scores(const AttnArgs& a, const int32_t* groups, const float* LSE, float* S,
-                cudaStream_t st);
+                int64_t row0, int64_t rows, cudaStream_t st);
 int simt_sparse(const AttnArgs& a, const int32_t* groups, const int32_t* indices,
                 const void* O_full, float* R_out, const float* R_in, void* O_out,
                 cudaStream_t st);
@@ -67,13 +68,15 @@ int tc_dense(const AttnArgs& a, void* O, float* lse, cudaStream_t st);
 
 // attn_tc_scores.cu: exact group scores on the tensor cores (bf16, d = 128, g_s <= 128)
 bool tc_scores_supported(const AttnArgs& a);
-int tc_scores(const AttnArgs& a, const int32_t* groups, const float* lse, float* S,
-              cudaStream_t st);
+int tc_scores(const AttnArgs& a, const int32_t* groups, const float* lse, float* S, int64_t row0,
+              int64_t rows, cudaStream_t st);
 
+// Exact group scores of the (head, group) rows row0 .. row0 + rows - 1 (row
+// = head * G + group) into S[0 .. rows * n_kv).
 inline int scores_pass(const AttnArgs& a, const int32_t* groups, const float* lse, float* S,
-                       cudaStream_t st) {
-  if (tc_scores_supported(a)) return tc_scores(a, groups, lse, S, st);
-  return simt_scores(a, groups, lse, S, st);
+                       int64_t row0, int64_t rows, cudaStream_t st) {
+  if (tc_scores_supported(a)) return tc_scores(a, groups, lse, S, row0, rows, st);
+  return simt_scores(a, groups, lse, S, row0, rows, st);
 }
 
 // Sparse pass with the residual epilogue on the best kernel for the shape.

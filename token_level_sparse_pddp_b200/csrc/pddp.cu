@@ -773,21 +773,16 @@ static int run_pddp_t(const T* Q, int64_t BH, int n_q, int gs, int32_t* groups, 
   const int64_t total = BH * n_q;
   pddp_init_kernel<<<(unsigned)ceil_div(total, 256), 256, 0, st>>>(w.perm, n_q, total);
   TLSP_TRY(check_launch());
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sm_count();
   if (kTc) {
-    cudaFuncSetAttribute(pddp_gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)kGramSmem);
-    cudaFuncSetAttribute(pddp_direction_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)kGramSmem);
+    TLSP_TRY(ensure_smem_limit((const void*)pddp_gram_tc_kernel, (int)kGramSmem));
+    TLSP_TRY(ensure_smem_limit((const void*)pddp_direction_tc_kernel, (int)kGramSmem));
   }
-  cudaFuncSetAttribute(pddp_split_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)((size_t)kSplitSmemKeys * 4));
+  TLSP_TRY(ensure_smem_limit((const void*)pddp_split_smem_kernel,
+                             (int)((size_t)kSplitSmemKeys * 4)));
   if (!kTc) {
-    cudaFuncSetAttribute(pddp_direction_kernel<T, D>,
-                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)direction_smem_bytes<D>());
+    TLSP_TRY(ensure_smem_limit((const void*)pddp_direction_kernel<T, D>,
+                               (int)direction_smem_bytes<D>()));
   }
   for (int level = 0; level < L; ++level) {
     const int64_t nodes = 1 << level;

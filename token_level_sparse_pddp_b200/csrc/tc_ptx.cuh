@@ -82,19 +82,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void* tmap, int 
       : "memory");
 }
 
-// Four rows r0..r3 x one box of columns starting at col of a 2-D tensor map
-// (box one row high) into four consecutive box rows at dst; completion is
-// counted in bytes on bar. Rows outside the tensor are filled with zeros.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const void* tmap, int col, int r0,
-                                            int r1, int r2, int r3, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3),
-      "r"(smem_u32(bar))
-      : "memory");
-}
-
 // Untiled bulk copy of `bytes` (a multiple of 16; both addresses 16-byte
 // aligned) from global to this CTA's shared memory; completion is counted in
 // bytes on bar.
@@ -203,6 +190,16 @@ __device__ __forceinline__ void reg_barrier(uint32_t (&r)[32]) {
         "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]),
         "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]),
         "+r"(r[31])
+      :
+      : "memory");
+}
+// reg_barrier for a 16-register TMEM load.
+__device__ __forceinline__ void reg_barrier16(uint32_t (&r)[16]) {
+  asm volatile(
+      ""
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+        "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
       :
       : "memory");
 }

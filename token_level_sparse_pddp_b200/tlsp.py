@@ -148,12 +148,19 @@ def launch_count() -> int:
 class Workspace:
     """Caller-owned scratch for the library calls (a zeroed torch byte tensor)."""
 
-    def __init__(self, dims: Dims, group_size: int, k: int, device=None):
-        n = lib().tlsp_workspace_bytes(ctypes.byref(dims), group_size, k)
+    def __init__(self, dims: Optional[Dims], group_size: int = 1, k: int = 1, device=None,
+                 nbytes: Optional[int] = None):
+        n = nbytes if nbytes is not None else lib().tlsp_workspace_bytes(
+            ctypes.byref(dims), group_size, k)
         if n == 0:
             raise TlspError(TLSP_ERR_INVALID_ARG, "tlsp_workspace_bytes")
         self.nbytes = n
         self.buf = torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+    @classmethod
+    def status_only(cls, device=None) -> "Workspace":
+        """The 256-byte workspace that the reuse step needs (its status word only)."""
+        return cls(None, nbytes=256, device=device)
 
     @property
     def ptr(self):
