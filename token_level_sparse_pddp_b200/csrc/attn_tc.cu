@@ -38,6 +38,9 @@
 // [0, n_q) before the ragged tail of the last group, or one other than -1
 // inside it, is recorded as TLSP_ERR_DEVICE_ASSERT (that key is read as a
 // zero row, that query row is skipped); such a tile's output is unspecified.
+#include <climits>
+#include <type_traits>
+
 #include "kernels.h"
 #include "tc_ptx.cuh"
 
@@ -171,21 +174,24 @@ __device__ __forceinline__ void gather_rows(uint32_t dst, const __nv_bfloat16* s
   }
 }
 
+// Marks positions past k in chunk_rows (no stored entry has this value).
+constexpr int kPastK = INT_MIN;
+
 // Global rows of chunk j of the selection for a producer thread of NT: read
-// from shared memory at sel_smem when the selection was staged there (an
-// explicit shared load), else from global memory at sel. Positions past k
-// are padding (-1); a selected entry outside [0, n_kv) is recorded and read
-// as a zero row.
-template <int NT>
-__device__ __forceinline__ void chunk_rows(const int32_t* sel, uint32_t sel_smem, bool staged,
-                                           int j, int k, int n_kv, int pt,
-                                           int (&rows)[2048 / NT], int* status) {
+// from shared memory at sel_smem when the selection was staged there
+// (kStaged; an explicit shared load), else from global memory at sel.
+// Positions past k are padding (-1); a selected entry outside [0, n_kv) is
+// recorded and read as a zero row.
+template <int NT, bool kStaged>
+__device__ __forceinline__ void chunk_rows(const int32_t* sel, uint32_t sel_smem, int j, int k,
+                                           int n_kv, int pt, int (&rows)[2048 / NT],
+                                           int* status) {
 #pragma unroll
   for (int it = 0; it < 2048 / NT; ++it) {
     const int q = j * kTile + it * (NT / 16) + (pt >> 4);
-    int v = -1;
+    int v = kPastK;
     if (q < k) {
-      if (staged)
+      if (kStaged)
         asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(sel_smem + 4u * (uint32_t)q));
       else
         v = __ldg(sel + q);
@@ -194,9 +200,8 @@ __device__ __forceinline__ void chunk_rows(const int32_t* sel, uint32_t sel_smem
   }
 #pragma unroll
   for (int it = 0; it < 2048 / NT; ++it) {
-    const int q = j * kTile + it * (NT / 16) + (pt >> 4);
-    if (q < k && (unsigned)rows[it] >= (unsigned)n_kv) {
-      record_status(status, TLSP_ERR_DEVICE_ASSERT);
+    if ((unsigned)rows[it] >= (unsigned)n_kv) {  // padding past k, or a bad entry
+      if (rows[it] != kPastK) record_status(status, TLSP_ERR_DEVICE_ASSERT);
       rows[it] = -1;
     }
   }
@@ -300,19 +305,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t slot0 = base + (is_k ? kSmK : kSmV);
       uint64_t* full = is_k ? bars.k_full : bars.v_full;
       uint64_t* empty = is_k ? bars.k_empty : bars.v_empty;
-      int rows[16];
-      chunk_rows<128>(sel, base + kSmIdx, idx_smem, 0, p.k, p.n_kv, qt, rows, p.status);
-      for (int j = 0; j < n_chunks; ++j) {
-        const int s = j % nslots, u = j / nslots;
-        if (u > 0 && !ptx::mbar_wait(&empty[s], (u - 1) & 1, abort_flag, kWaitNs)) {
-          fail(bars, p.status);
-          break;
+      // the chunk loop, with the selection read from shared memory (staged)
+      // or from global memory, chosen once
+      auto stream = [&](auto staged) {
+        constexpr bool kStaged = decltype(staged)::value;
+        int rows[16];
+        chunk_rows<128, kStaged>(sel, base + kSmIdx, 0, p.k, p.n_kv, qt, rows, p.status);
+        for (int j = 0; j < n_chunks; ++j) {
+          const int s = j % nslots, u = j / nslots;
+          if (u > 0 && !ptx::mbar_wait(&empty[s], (u - 1) & 1, abort_flag, kWaitNs)) {
+            fail(bars, p.status);
+            break;
+          }
+          gather_rows<128>(slot0 + s * kTileBytes, src, rows, qt);
+          ptx::cp_async_arrive_noinc(&full[s]);
+          if (j + 1 < n_chunks)
+            chunk_rows<128, kStaged>(sel, base + kSmIdx, j + 1, p.k, p.n_kv, qt, rows, p.status);
         }
-        gather_rows<128>(slot0 + s * kTileBytes, src, rows, qt);
-        ptx::cp_async_arrive_noinc(&full[s]);
-        if (j + 1 < n_chunks)
-          chunk_rows<128>(sel, base + kSmIdx, idx_smem, j + 1, p.k, p.n_kv, qt, rows, p.status);
-      }
+      };
+      if (idx_smem)
+        stream(std::true_type{});
+      else
+        stream(std::false_type{});
       }
       if (pt < 128 && p.wave > 0 && (int64_t)blockIdx.x + p.wave < (int64_t)gridDim.x)
         warm_tile_l2<kMode>(p, (int64_t)blockIdx.x + p.wave, pt);
@@ -370,7 +384,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ softmax
     const int r = tid;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    const int tok = group_token(grp, t * kTile + r, members, p);
+    // (the producers' Q gather validates the group entries and records bad
+    // ones; here a bad entry, or anything in the ragged tail, is skipped)
+    const int gr = t * kTile + r;
+    int tok = gr < members ? grp[gr] : -1;
+    if (tok >= p.n_q) tok = -1;
     if (tok >= 0) {  // the row the epilogue reads, towards L2 while the tile computes
       const int64_t row = (bh * p.n_q + tok) * kD;
       if (kMode == kReuse) {
