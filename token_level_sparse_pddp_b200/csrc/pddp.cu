@@ -118,18 +118,18 @@ __device__ void chunk_moments(const T* __restrict__ X, const int32_t* __restrict
 template <class T, int D>
 __global__ void __launch_bounds__(kMomThreads)
 pddp_moments_kernel(const T* __restrict__ Q, const int32_t* __restrict__ perm, int n_q, int gs,
-                    int G, int level, int cpn, float* __restrict__ partials) {
+                    int G, int level, int cpn, int bh0, float* __restrict__ partials) {
   constexpr int BLK = D / 16;
   __shared__ float s_rows[kStageRows * D];
   __shared__ float s_mu[D];
   __shared__ float s_red[kMomThreads];
-  const int j = blockIdx.y, bh = blockIdx.z, c = blockIdx.x;
+  const int j = blockIdx.y, hl = blockIdx.z, bh = bh0 + hl, c = blockIdx.x;
   const NodeDesc nd = node_at(n_q, gs, G, level, j);
   if (!nd.active) return;
   const int len = (nd.cnt + cpn - 1) / cpn;
   const int begin = nd.off + c * len;
   const int end = min(nd.off + nd.cnt, begin + len);
-  float* rec = partials + ((int64_t)(bh * (1 << level) + j) * cpn + c) * Moments<D>::kStride;
+  float* rec = partials + ((int64_t)(hl * (1 << level) + j) * cpn + c) * Moments<D>::kStride;
   if (begin >= end) {  // empty chunk: count 0
     if (threadIdx.x == 0) rec[Moments<D>::kN] = 0.f;
     return;
@@ -153,13 +153,13 @@ pddp_moments_kernel(const T* __restrict__ Q, const int32_t* __restrict__ perm, i
 // own entry, so the in-place update has no race.
 template <int D>
 __global__ void __launch_bounds__(256)
-pddp_reduce_kernel(int n_q, int gs, int G, int level, int cpn, float* __restrict__ partials,
-                   float* __restrict__ node_mu) {
+pddp_reduce_kernel(int n_q, int gs, int G, int level, int cpn, int bh0,
+                   float* __restrict__ partials, float* __restrict__ node_mu) {
   __shared__ float s_mu[D];
-  const int slice = blockIdx.x, j = blockIdx.y, bh = blockIdx.z, t = threadIdx.x;
+  const int slice = blockIdx.x, j = blockIdx.y, hl = blockIdx.z, bh = bh0 + hl, t = threadIdx.x;
   const NodeDesc nd = node_at(n_q, gs, G, level, j);
   if (!nd.active) return;
-  float* recs = partials + (int64_t)(bh * (1 << level) + j) * cpn * Moments<D>::kStride;
+  float* recs = partials + (int64_t)(hl * (1 << level) + j) * cpn * Moments<D>::kStride;
   if (t < D) {
     float s = 0.f, n = 0.f;
     for (int c = 0; c < cpn; ++c) {
@@ -196,7 +196,7 @@ constexpr size_t direction_smem_bytes() {
 template <class T, int D>
 __global__ void __launch_bounds__(kMomThreads)
 pddp_direction_kernel(const T* __restrict__ Q, const int32_t* __restrict__ perm, int n_q, int gs,
-                      int G, int level, int cpn, const float* __restrict__ partials,
+                      int G, int level, int cpn, int bh0, const float* __restrict__ partials,
                       float* __restrict__ node_mu, float* __restrict__ node_v) {
   constexpr int BLK = D / 16;
   extern __shared__ float smem[];
@@ -207,7 +207,7 @@ pddp_direction_kernel(const T* __restrict__ Q, const int32_t* __restrict__ perm,
   float* s_w = s_v + D;                   // D
   float* s_red = s_w + D + D;             // kMomThreads
   float* s_misc = s_red + kMomThreads;    // 8
-  const int j = blockIdx.x, bh = blockIdx.y, t = threadIdx.x;
+  const int j = blockIdx.x, hl = blockIdx.y, bh = bh0 + hl, t = threadIdx.x;
   const NodeDesc nd = node_at(n_q, gs, G, level, j);
   if (!nd.active) return;
   const int bi = t / 16, bj = t % 16;
@@ -216,7 +216,7 @@ pddp_direction_kernel(const T* __restrict__ Q, const int32_t* __restrict__ perm,
     chunk_moments<T, D>(Q + (int64_t)bh * n_q * D, perm + (int64_t)bh * n_q, nd.off,
                         nd.off + nd.cnt, s_rows, s_mu, s_red, acc);
   } else {  // scatter and mean combined by pddp_reduce_kernel (record 0, node_mu)
-    const float* rec = partials + (int64_t)(bh * (1 << level) + j) * cpn * Moments<D>::kStride;
+    const float* rec = partials + (int64_t)(hl * (1 << level) + j) * cpn * Moments<D>::kStride;
     if (t < D) s_mu[t] = node_mu[((int64_t)bh * G + j) * D + t];
 #pragma unroll
     for (int i = 0; i < BLK; ++i)
@@ -599,18 +599,18 @@ __device__ __forceinline__ void gram_row_part(uint32_t tmem, const GramShared& s
 // Chunk records of the tensor-core path (same format as pddp_moments_kernel).
 __global__ void __launch_bounds__(kGT, 2)
 pddp_gram_tc_kernel(const __nv_bfloat16* __restrict__ Q, const int32_t* __restrict__ perm,
-                    int n_q, int gs, int G, int level, int cpn, float* __restrict__ partials,
-                    int* status) {
+                    int n_q, int gs, int G, int level, int cpn, int bh0,
+                    float* __restrict__ partials, int* status) {
   extern __shared__ uint8_t smem_raw[];
   const GramCta cta = gram_cta_layout(smem_raw);
   GramShared& sh = *cta.sh;
-  const int c = blockIdx.x, j = blockIdx.y, bh = blockIdx.z, t = threadIdx.x;
+  const int c = blockIdx.x, j = blockIdx.y, hl = blockIdx.z, bh = bh0 + hl, t = threadIdx.x;
   const NodeDesc nd = node_at(n_q, gs, G, level, j);
   if (!nd.active) return;
   const int len = (nd.cnt + cpn - 1) / cpn;
   const int begin = nd.off + c * len;
   const int end = min(nd.off + nd.cnt, begin + len);
-  float* rec = partials + ((int64_t)(bh * (1 << level) + j) * cpn + c) * Moments<kGD>::kStride;
+  float* rec = partials + ((int64_t)(hl * (1 << level) + j) * cpn + c) * Moments<kGD>::kStride;
   if (begin >= end) {
     if (t == 0) rec[Moments<kGD>::kN] = 0.f;
     return;
@@ -641,13 +641,14 @@ pddp_gram_tc_kernel(const __nv_bfloat16* __restrict__ Q, const int32_t* __restri
 // channel on ties) positive.
 __global__ void __launch_bounds__(kGT, 2)
 pddp_direction_tc_kernel(const __nv_bfloat16* __restrict__ Q, const int32_t* __restrict__ perm,
-                         int n_q, int gs, int G, int level, int cpn,
+                         int n_q, int gs, int G, int level, int cpn, int bh0,
                          const float* __restrict__ partials, float* __restrict__ node_mu,
                          float* __restrict__ node_v, int* status) {
   extern __shared__ uint8_t smem_raw[];
   const GramCta cta = gram_cta_layout(smem_raw);
   GramShared& sh = *cta.sh;
-  const int j = blockIdx.x, bh = blockIdx.y, t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int j = blockIdx.x, hl = blockIdx.y, bh = bh0 + hl, t = threadIdx.x, warp = t >> 5,
+            lane = t & 31;
   const NodeDesc nd = node_at(n_q, gs, G, level, j);
   if (!nd.active) return;
   const int a = 32 * (warp & 3) + lane, e0 = 64 * (warp >> 2);
@@ -665,7 +666,7 @@ pddp_direction_tc_kernel(const __nv_bfloat16* __restrict__ Q, const int32_t* __r
     if (!ok) return;
   } else {
     const float4* src = reinterpret_cast<const float4*>(
-        partials + (int64_t)(bh * (1 << level) + j) * cpn * Moments<kGD>::kStride + a * kGD + e0);
+        partials + (int64_t)(hl * (1 << level) + j) * cpn * Moments<kGD>::kStride + a * kGD + e0);
 #pragma unroll
     for (int e = 0; e < 64; e += 4) {
       const float4 u = src[e / 4];
@@ -758,6 +759,9 @@ __global__ void pddp_emit_kernel(const int32_t* __restrict__ perm, int n_q, int 
 
 // ----------------------------------------------------------------- host side
 
+// Chunk records per head and tree level at most (see run_pddp_t).
+constexpr int64_t kChunksPerHead = 32;
+
 static int levels_of(int G) {
   int L = 0;
   while ((1 << L) < G) ++L;
@@ -773,7 +777,6 @@ static int run_pddp_t(const T* Q, int64_t BH, int n_q, int gs, int32_t* groups, 
   const int64_t total = BH * n_q;
   pddp_init_kernel<<<(unsigned)ceil_div(total, 256), 256, 0, st>>>(w.perm, n_q, total);
   TLSP_TRY(check_launch());
-  const int sms = device_sm_count();
   if (kTc) {
     TLSP_TRY(ensure_smem_limit((const void*)pddp_gram_tc_kernel, (int)kGramSmem));
     TLSP_TRY(ensure_smem_limit((const void*)pddp_direction_tc_kernel, (int)kGramSmem));
@@ -787,37 +790,45 @@ static int run_pddp_t(const T* Q, int64_t BH, int n_q, int gs, int32_t* groups, 
   for (int level = 0; level < L; ++level) {
     const int64_t nodes = 1 << level;
     const int64_t max_rows = ceil_div(n_q, nodes) + gs;
-    // Tensor-core path: about two resident CTAs per SM over all chunks, each
-    // chunk at least two MMA batches. SIMT path: chunks of about 256 rows.
-    int64_t cpn = kTc ? std::min<int64_t>(ceil_div(2 * (int64_t)sms, BH * nodes),
-                                          ceil_div(max_rows, 2 * kSub))
-                      : ceil_div(max_rows, 256);
-    cpn = std::min<int64_t>(cpn, w.partial_slots / (BH * nodes));
+    // Chunks per node depend only on the node sizes (never on how many heads
+    // the call holds or on the device), so a head's groups are the same
+    // whether it is grouped alone or with others: at most kChunksPerHead
+    // records per head and level, each chunk at least two MMA batches (tensor
+    // cores) or about 256 rows (SIMT).
+    int64_t cpn = kTc ? ceil_div(max_rows, 2 * kSub) : ceil_div(max_rows, 256);
+    cpn = std::min<int64_t>(cpn, std::max<int64_t>(1, kChunksPerHead / nodes));
     if (cpn < 2) cpn = 1;
-    if (cpn > 1) {
-      const dim3 grid((unsigned)cpn, (unsigned)nodes, (unsigned)BH);
+    // heads whose chunk records fit in the workspace at once
+    const int64_t hb = cpn > 1 ? std::max<int64_t>(1, w.partial_slots / (nodes * cpn)) : BH;
+    for (int64_t h0 = 0; h0 < BH; h0 += hb) {
+      const unsigned nh = (unsigned)std::min<int64_t>(hb, BH - h0);
+      if (cpn > 1) {
+        const dim3 grid((unsigned)cpn, (unsigned)nodes, nh);
+        if constexpr (kTc) {
+          pddp_gram_tc_kernel<<<grid, kGT, kGramSmem, st>>>(Q, w.perm, n_q, gs, G, level,
+                                                            (int)cpn, (int)h0, w.partials,
+                                                            w.status);
+        } else {
+          pddp_moments_kernel<T, D><<<grid, kMomThreads, 0, st>>>(Q, w.perm, n_q, gs, G, level,
+                                                                  (int)cpn, (int)h0, w.partials);
+        }
+        TLSP_TRY(check_launch());
+        pddp_reduce_kernel<D><<<dim3(D * D / 256, (unsigned)nodes, nh), 256, 0, st>>>(
+            n_q, gs, G, level, (int)cpn, (int)h0, w.partials, w.node_mu);
+        TLSP_TRY(check_launch());
+      }
       if constexpr (kTc) {
-        pddp_gram_tc_kernel<<<grid, kGT, kGramSmem, st>>>(Q, w.perm, n_q, gs, G, level, (int)cpn,
-                                                          w.partials, w.status);
+        pddp_direction_tc_kernel<<<dim3((unsigned)nodes, nh), kGT,
+                                   cpn > 1 ? kDirSmemNoGram : kGramSmem, st>>>(
+            Q, w.perm, n_q, gs, G, level, (int)cpn, (int)h0, w.partials, w.node_mu, w.node_v,
+            w.status);
       } else {
-        pddp_moments_kernel<T, D><<<grid, kMomThreads, 0, st>>>(Q, w.perm, n_q, gs, G, level,
-                                                                (int)cpn, w.partials);
+        pddp_direction_kernel<T, D><<<dim3((unsigned)nodes, nh), kMomThreads,
+                                      direction_smem_bytes<D>(), st>>>(
+            Q, w.perm, n_q, gs, G, level, (int)cpn, (int)h0, w.partials, w.node_mu, w.node_v);
       }
       TLSP_TRY(check_launch());
-      pddp_reduce_kernel<D><<<dim3(D * D / 256, (unsigned)nodes, (unsigned)BH), 256, 0, st>>>(
-          n_q, gs, G, level, (int)cpn, w.partials, w.node_mu);
-      TLSP_TRY(check_launch());
     }
-    if constexpr (kTc) {
-      pddp_direction_tc_kernel<<<dim3((unsigned)nodes, (unsigned)BH), kGT,
-                                 cpn > 1 ? kDirSmemNoGram : kGramSmem, st>>>(
-          Q, w.perm, n_q, gs, G, level, (int)cpn, w.partials, w.node_mu, w.node_v, w.status);
-    } else {
-      pddp_direction_kernel<T, D><<<dim3((unsigned)nodes, (unsigned)BH), kMomThreads,
-                                    direction_smem_bytes<D>(), st>>>(
-          Q, w.perm, n_q, gs, G, level, (int)cpn, w.partials, w.node_mu, w.node_v);
-    }
-    TLSP_TRY(check_launch());
     constexpr int kRowsPerBlock = 256 / (D * (int)sizeof(T) / 16) * kProjRows;
     pddp_project_kernel<T, D>
         <<<dim3((unsigned)ceil_div(n_q, kRowsPerBlock), (unsigned)BH), 256, 0, st>>>(
