@@ -27,11 +27,16 @@
 // buffer [0,256), O [256,384), P double buffer [384,512). K has three
 // shared-memory slots and V two, so loads run ahead of the math.
 // The softmax keeps a reference max per row and computes each chunk in one
-// pass against it; only when a chunk's max exceeds the reference by more than
-// 2^8 is the reference raised, O rescaled in TMEM and the chunk recomputed
-// (by the whole warp: its TMEM accesses are warp-collective).
+// pass against it (the first chunk's reference is the max of its first 32
+// columns); only when a chunk's max exceeds the reference by more than 2^8 is
+// the reference raised, O rescaled in TMEM and the chunk recomputed (by the
+// whole warp: its TMEM accesses are warp-collective).
 // Between raises the stale reference is used for numerator and denominator
 // alike, which cancels exactly in O / l.
+// Epilogue operands (R rows for the reuse step, O_full rows for the anchor
+// step) are copied by the producers into the two K slots that the last chunk
+// does not use, once those slots' last QK^T has completed, so the epilogue
+// reads them from shared memory instead of waiting on L2 per row.
 // Every wait is bounded (1 s); on expiry the kernel records
 // TLSP_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 // Index checks: a selection entry outside [0, n_kv), a group entry outside
@@ -71,7 +76,7 @@ struct Bars {
   uint64_t q_full;
   uint64_t k_full[kKSlots], k_empty[kKSlots], v_full[kVSlots], v_empty[kVSlots];
   uint64_t s_full[2], p_full[2];
-  uint64_t o_done, o_final, drain;
+  uint64_t o_done, o_final, drain, r_full;
   uint32_t tmem_base;
   int abort;
 };
@@ -207,6 +212,33 @@ __device__ __forceinline__ void chunk_rows(const int32_t* sel, uint32_t sel_smem
   }
 }
 
+// The two K slots that the last of n_chunks chunks does not use (ascending):
+// they hold the epilogue's operand rows.
+__device__ __forceinline__ void epi_slots(int n_chunks, int& a, int& b) {
+  const int last = (n_chunks - 1) % kKSlots;
+  a = last == 0 ? 1 : 0;
+  b = last == 2 ? 1 : 2;
+}
+
+// The last chunk before the final one that used K slot s, or -1.
+__device__ __forceinline__ int last_use(int s, int n_chunks) {
+  const int m = n_chunks - 2;
+  if (m < s) return -1;
+  return m - (m - s) % kKSlots;
+}
+
+// Shared-memory address of 16-byte chunk c of epilogue row r: reuse rows are
+// R's 512 bytes (rows 0-63 in slot a, 64-127 in slot b), anchor rows are
+// O_full's 256 bytes (all in slot a). Chunk c sits at position c ^ (r mod 8)
+// of its row, so eight consecutive rows reading the same c hit eight
+// different 16-byte bank groups.
+template <int kMode>
+__device__ __forceinline__ uint32_t epi_addr(uint32_t slot_a, uint32_t slot_b, int r, int c) {
+  const uint32_t sw = (uint32_t)(c ^ (r & 7)) << 4;
+  if (kMode == kReuse) return (r < 64 ? slot_a : slot_b) + (uint32_t)(r & 63) * 512u + sw;
+  return slot_a + (uint32_t)r * 256u + sw;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -257,6 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(&bars.o_done, 1);
     ptx::mbar_init(&bars.o_final, 1);
     ptx::mbar_init(&bars.drain, 1);
+    ptx::mbar_init(&bars.r_full, 256);
     bars.abort = 0;
     ptx::fence_mbar_init();
   }
@@ -330,6 +363,41 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (pt < 128 && p.wave > 0 && (int64_t)blockIdx.x + p.wave < (int64_t)gridDim.x)
         warm_tile_l2<kMode>(p, (int64_t)blockIdx.x + p.wave, pt);
+      // Epilogue operand rows into the two K slots the last chunk does not
+      // use, once their last QK^T has completed (by then every earlier phase
+      // of those slots' barriers has completed too, for K and V producers
+      // alike, so the parity waits are unambiguous). A warp instruction moves
+      // one whole R row (reuse) or two O_full rows (anchor).
+      {
+        int sa, sb;
+        epi_slots(n_chunks, sa, sb);
+        bool ok = true;
+        for (int i = 0; i < 2 && ok; ++i) {
+          const int s = i ? sb : sa, jl = last_use(s, n_chunks);
+          if (jl >= 0 && !ptx::mbar_wait(&bars.k_empty[s], (jl / kKSlots) & 1, abort_flag, kWaitNs))
+            ok = false;
+        }
+        if (!ok) {
+          fail(bars, p.status);
+        } else {
+          const uint32_t slot_a = base + kSmK + sa * kTileBytes, slot_b = base + kSmK + sb * kTileBytes;
+          constexpr int kChunks = kMode == kReuse ? 32 : 16;  // 16-byte chunks per row
+          constexpr int kRowsPerPass = 256 / kChunks;
+#pragma unroll 4
+          for (int it = 0; it < kTile / kRowsPerPass; ++it) {
+            const int r = it * kRowsPerPass + pt / kChunks, c = pt % kChunks;
+            const int gr = t * kTile + r;
+            int tok = gr < members ? __ldg(grp + gr) : -1;
+            if (tok >= p.n_q) tok = -1;
+            if (tok < 0) continue;
+            const int64_t row = (bh * p.n_q + tok) * kD;
+            const void* src = kMode == kReuse ? (const void*)(p.R_in + row + c * 4)
+                                              : (const void*)(p.O_full + row + c * 8);
+            ptx::cp_async16(epi_addr<kMode>(slot_a, slot_b, r, c), src, 16u);
+          }
+          ptx::cp_async_arrive_noinc(&bars.r_full);
+        }
+      }
       ptx::cp_async_wait_all();
     }
   } else if (warp == 12) {
@@ -461,29 +529,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         max_out = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       };
       float sum, mx;
-      bool raise = (j == 0);
-      if (!raise) {
-        p_pass(m_run, sum, mx);  // speculative: usually the reference max still holds
-        // the rescale below is made of warp-collective TMEM accesses, so the
-        // warp takes it together when any of its rows needs it
-        raise = __any_sync(0xffffffffu, mx * p.scale_log2 > m_run + kRescaleLog2);
-      } else {
-        // first chunk: its max becomes the reference
+      if (j == 0) {
+        // first chunk: the max of its first 32 columns becomes the reference
+        uint32_t c[32];
+        ptx::tmem_ld32(s_col, c);
+        ptx::tmem_ld_wait(c);
         float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-        for (int b = 0; b < 4; ++b) {
-          uint32_t c[32];
-          ptx::tmem_ld32(s_col + 32 * b, c);
-          ptx::tmem_ld_wait(c);
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (32 * b + e < valid_n) pm[e & 3] = fmaxf(pm[e & 3], __uint_as_float(c[e]));
-        }
-        mx = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
+        for (int e = 0; e < 32; ++e)
+          if (e < valid_n) pm[e & 3] = fmaxf(pm[e & 3], __uint_as_float(c[e]));
+        m_run = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])) * p.scale_log2;
       }
+      p_pass(m_run, sum, mx);  // speculative: usually the reference max still holds
+      // the rescale below is made of warp-collective TMEM accesses, so the
+      // warp takes it together when any of its rows needs it
+      const bool raise = __any_sync(0xffffffffu, mx * p.scale_log2 > m_run + kRescaleLog2);
       if (raise) {
         // rows of the warp that do not need it keep their reference (factor 1)
-        const float m_tile = j > 0 ? fmaxf(mx * p.scale_log2, m_run) : mx * p.scale_log2;
+        const float m_tile = fmaxf(mx * p.scale_log2, m_run);
         if (j > 0) {
           // raise the reference max: O *= 2^(m_run - m_tile) once PV(j-1) has landed
           const float f = ptx::ex2(m_run - m_tile);
@@ -513,25 +576,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_arrive(&bars.p_full[s]);
     }
     const int64_t row = (bh * p.n_q + (tok >= 0 ? tok : 0)) * kD;
-    // Epilogue operands (R rows for the reuse step, O_full rows for the anchor
-    // step) are read one 32-column block ahead: block 0 before the final wait,
-    // block q + 1 while block q's TMEM load is in flight.
+    // Epilogue: O / l from TMEM, 32 columns at a time, with the operand row
+    // (R for the reuse step, O_full for the anchor step) from shared memory.
     const bool has_row = tok >= 0;
-    float4 rb[2][8];  // reuse: R, 32 fp32 columns per block
-    uint4 ob[2][4];   // anchor: O_full, 32 bf16 columns per block
-    auto load_block = [&](int q, int b) {
-      if (kMode == kReuse) {
-        const float4* rs = reinterpret_cast<const float4*>(p.R_in + row + q * 32);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) rb[b][c] = rs[c];
-      } else if (kMode == kAnchor) {
-        const uint4* os = reinterpret_cast<const uint4*>(p.O_full + row + q * 32);
-#pragma unroll
-        for (int c = 0; c < 4; ++c) ob[b][c] = os[c];
-      }
-    };
-    if (has_row) load_block(0, 0);
+    int sa, sb;
+    epi_slots(n_chunks, sa, sb);
+    const uint32_t slot_a = base + kSmK + sa * kTileBytes, slot_b = base + kSmK + sb * kTileBytes;
     if (ok && !ptx::mbar_wait(&bars.o_final, 0, abort_flag, kWaitNs)) ok = false;
+    if (ok && !ptx::mbar_wait(&bars.r_full, 0, abort_flag, kWaitNs)) ok = false;
     if (!ok) {
       fail(bars, p.status);
     } else {
@@ -541,7 +593,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int q = 0; q < 4; ++q) {
         uint32_t o[32];
         ptx::tmem_ld32(tl + kTmO + q * 32, o);
-        if (has_row && q < 3) load_block(q + 1, (q + 1) & 1);
         ptx::tmem_ld_wait(o);
         if (!has_row) continue;  // (no warp-collective instruction follows in this iteration)
         const int c0 = q * 32;
@@ -549,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float4* dst = reinterpret_cast<float4*>(p.R_out + row + c0);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            const uint4 u = ob[q & 1][c];
+            const uint4 u = ptx::ld_shared_v4(epi_addr<kMode>(slot_a, slot_b, r, 4 * q + c));
             const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
@@ -565,18 +616,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint4* dst = reinterpret_cast<uint4*>(p.O_out + row + c0);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            const float4 r0 = kMode == kReuse ? rb[q & 1][2 * c] : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float4 r1 =
-                kMode == kReuse ? rb[q & 1][2 * c + 1] : make_float4(0.f, 0.f, 0.f, 0.f);
+            const uint4 u0 = ptx::ld_shared_v4(epi_addr<kMode>(slot_a, slot_b, r, 8 * q + 2 * c));
+            const uint4 u1 = ptx::ld_shared_v4(epi_addr<kMode>(slot_a, slot_b, r, 8 * q + 2 * c + 1));
             uint4 out;
-            out.x = pack_bf16(__uint_as_float(o[8 * c]) * inv + r0.x,
-                              __uint_as_float(o[8 * c + 1]) * inv + r0.y);
-            out.y = pack_bf16(__uint_as_float(o[8 * c + 2]) * inv + r0.z,
-                              __uint_as_float(o[8 * c + 3]) * inv + r0.w);
-            out.z = pack_bf16(__uint_as_float(o[8 * c + 4]) * inv + r1.x,
-                              __uint_as_float(o[8 * c + 5]) * inv + r1.y);
-            out.w = pack_bf16(__uint_as_float(o[8 * c + 6]) * inv + r1.z,
-                              __uint_as_float(o[8 * c + 7]) * inv + r1.w);
+            out.x = pack_bf16(__uint_as_float(o[8 * c]) * inv + __uint_as_float(u0.x),
+                              __uint_as_float(o[8 * c + 1]) * inv + __uint_as_float(u0.y));
+            out.y = pack_bf16(__uint_as_float(o[8 * c + 2]) * inv + __uint_as_float(u0.z),
+                              __uint_as_float(o[8 * c + 3]) * inv + __uint_as_float(u0.w));
+            out.z = pack_bf16(__uint_as_float(o[8 * c + 4]) * inv + __uint_as_float(u1.x),
+                              __uint_as_float(o[8 * c + 5]) * inv + __uint_as_float(u1.y));
+            out.w = pack_bf16(__uint_as_float(o[8 * c + 6]) * inv + __uint_as_float(u1.z),
+                              __uint_as_float(o[8 * c + 7]) * inv + __uint_as_float(u1.w));
             dst[c] = out;
           }
         }
