@@ -575,7 +575,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bars.p_full[s]);
     }
-    const int64_t row = (bh * p.n_q + (tok >= 0 ? tok : 0)) * kD;
     // Epilogue: O / l from TMEM, 32 columns at a time, with the operand row
     // (R for the reuse step, O_full for the anchor step) from shared memory.
     const bool has_row = tok >= 0;
@@ -584,20 +583,28 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t slot_a = base + kSmK + sa * kTileBytes, slot_b = base + kSmK + sb * kTileBytes;
     if (ok && !ptx::mbar_wait(&bars.o_final, 0, abort_flag, kWaitNs)) ok = false;
     if (ok && !ptx::mbar_wait(&bars.r_full, 0, abort_flag, kWaitNs)) ok = false;
+    ok = __all_sync(0xffffffffu, ok);  // the epilogue's TMEM loads and shuffles are warp-collective
     if (!ok) {
       fail(bars, p.status);
     } else {
       ptx::tc_fence_after();
       const float inv = 1.f / l_run;
+      // Each thread writes its output row (bf16 O for the reuse step, fp32 R
+      // for the anchor step) into the free V slots, chunk c of row r at
+      // position c ^ (r mod 8); each warp then stores its own 32 rows with
+      // whole-row warp instructions, so a store touches 2 (or 1) rows instead
+      // of 32.
+      const uint32_t ostage = base + kSmV;
+      constexpr uint32_t kRowBytes = kMode == kReuse ? 256u : 512u;
+      const uint32_t orow = ostage + (uint32_t)r * kRowBytes;
+      auto ost = [&](int c) { return orow + ((uint32_t)(c ^ (r & 7)) << 4); };
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t o[32];
         ptx::tmem_ld32(tl + kTmO + q * 32, o);
         ptx::tmem_ld_wait(o);
         if (!has_row) continue;  // (no warp-collective instruction follows in this iteration)
-        const int c0 = q * 32;
         if (kMode == kAnchor) {
-          float4* dst = reinterpret_cast<float4*>(p.R_out + row + c0);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const uint4 u = ptx::ld_shared_v4(epi_addr<kMode>(slot_a, slot_b, r, 4 * q + c));
@@ -605,31 +612,53 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const int e = 8 * c + 4 * h;
-              dst[2 * c + h] = make_float4(
-                  __uint_as_float(w[2 * h] << 16) - __uint_as_float(o[e]) * inv,
-                  __uint_as_float(w[2 * h] & 0xffff0000u) - __uint_as_float(o[e + 1]) * inv,
-                  __uint_as_float(w[2 * h + 1] << 16) - __uint_as_float(o[e + 2]) * inv,
-                  __uint_as_float(w[2 * h + 1] & 0xffff0000u) - __uint_as_float(o[e + 3]) * inv);
+              ptx::st_shared_v4(
+                  ost(8 * q + 2 * c + h),
+                  __float_as_uint(__uint_as_float(w[2 * h] << 16) - __uint_as_float(o[e]) * inv),
+                  __float_as_uint(__uint_as_float(w[2 * h] & 0xffff0000u) -
+                                  __uint_as_float(o[e + 1]) * inv),
+                  __float_as_uint(__uint_as_float(w[2 * h + 1] << 16) -
+                                  __uint_as_float(o[e + 2]) * inv),
+                  __float_as_uint(__uint_as_float(w[2 * h + 1] & 0xffff0000u) -
+                                  __uint_as_float(o[e + 3]) * inv));
             }
           }
         } else {
-          uint4* dst = reinterpret_cast<uint4*>(p.O_out + row + c0);
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
             const uint4 u0 = ptx::ld_shared_v4(epi_addr<kMode>(slot_a, slot_b, r, 8 * q + 2 * c));
             const uint4 u1 = ptx::ld_shared_v4(epi_addr<kMode>(slot_a, slot_b, r, 8 * q + 2 * c + 1));
-            uint4 out;
-            out.x = pack_bf16(__uint_as_float(o[8 * c]) * inv + __uint_as_float(u0.x),
-                              __uint_as_float(o[8 * c + 1]) * inv + __uint_as_float(u0.y));
-            out.y = pack_bf16(__uint_as_float(o[8 * c + 2]) * inv + __uint_as_float(u0.z),
-                              __uint_as_float(o[8 * c + 3]) * inv + __uint_as_float(u0.w));
-            out.z = pack_bf16(__uint_as_float(o[8 * c + 4]) * inv + __uint_as_float(u1.x),
-                              __uint_as_float(o[8 * c + 5]) * inv + __uint_as_float(u1.y));
-            out.w = pack_bf16(__uint_as_float(o[8 * c + 6]) * inv + __uint_as_float(u1.z),
-                              __uint_as_float(o[8 * c + 7]) * inv + __uint_as_float(u1.w));
-            dst[c] = out;
+            ptx::st_shared_v4(
+                ost(4 * q + c),
+                pack_bf16(__uint_as_float(o[8 * c]) * inv + __uint_as_float(u0.x),
+                          __uint_as_float(o[8 * c + 1]) * inv + __uint_as_float(u0.y)),
+                pack_bf16(__uint_as_float(o[8 * c + 2]) * inv + __uint_as_float(u0.z),
+                          __uint_as_float(o[8 * c + 3]) * inv + __uint_as_float(u0.w)),
+                pack_bf16(__uint_as_float(o[8 * c + 4]) * inv + __uint_as_float(u1.x),
+                          __uint_as_float(o[8 * c + 5]) * inv + __uint_as_float(u1.y)),
+                pack_bf16(__uint_as_float(o[8 * c + 6]) * inv + __uint_as_float(u1.z),
+                          __uint_as_float(o[8 * c + 7]) * inv + __uint_as_float(u1.w)));
           }
         }
+      }
+      __syncwarp();
+      // whole-row stores: lane l takes chunk l % kPer of row (l / kPer) of
+      // each group of 32 / kPer rows
+      constexpr int kPer = (int)(kRowBytes / 16);  // 16-byte chunks per row
+      constexpr int kRowsPer = 32 / kPer;
+#pragma unroll 4
+      for (int i = 0; i < 32 / kRowsPer; ++i) {
+        const int rl = i * kRowsPer + lane / kPer, c = lane % kPer;
+        const int rr = warp * 32 + rl;
+        const int tok_rr = __shfl_sync(0xffffffffu, tok, rl);
+        if (tok_rr < 0) continue;
+        const uint4 v = ptx::ld_shared_v4(ostage + (uint32_t)rr * kRowBytes +
+                                          ((uint32_t)(c ^ (rr & 7)) << 4));
+        const int64_t grow = (bh * p.n_q + tok_rr) * kD;
+        if (kMode == kAnchor)
+          reinterpret_cast<uint4*>(p.R_out + grow)[c] = v;
+        else
+          reinterpret_cast<uint4*>(p.O_out + grow)[c] = v;
       }
     }
   }
