@@ -127,6 +127,29 @@ def test_topk_fed_many_rows_and_shapes(T):
             assert np.array_equal(idx[r], orc.topk(S[r].astype(np.float64), k)), (n_kv, k, r)
 
 
+def test_topk_structured_rows(T):
+    # rows of 8K-64K keys with structure: a smooth field, sparse spikes, a
+    # ramp, ties at the k-th key, a third of the row at the max, signed zeros;
+    # every row must match the oracle
+    from oracle import oracle as orc
+    rng = np.random.default_rng(11)
+    for rows, n_kv, k in [(600, 32760, 1664), (8, 8192, 300), (8, 65536, 2000), (9, 20001, 1000)]:
+        S = rng.exponential(1.0, size=(rows, n_kv)).astype(np.float32) ** 3
+        S[0] = np.cumsum(rng.standard_normal(n_kv)).astype(np.float32)   # smooth field
+        S[1] = 0.0
+        S[1, 63::64] = 1.0 + rng.random(len(S[1, 63::64])).astype(np.float32)  # sparse spikes
+        S[2] = np.arange(n_kv, dtype=np.float32)[::-1]                       # ramp
+        S[3] = np.round(S[3] * 4) / 4                                        # ties at the k-th key
+        S[4, ::3] = S[4].max()                                               # a third of the row at the max
+        S[5, 1::2] = -0.0
+        S[5, ::2] = 0.0
+        S[6] = rng.standard_normal(n_kv).astype(np.float32)
+        idx = T.topk_from_scores(torch.from_numpy(S).cuda(), k).cpu().numpy()
+        check = range(rows) if rows <= 16 else list(range(10)) + list(range(rows - 10, rows))
+        for r in check:
+            assert np.array_equal(idx[r], orc.topk(S[r].astype(np.float64), k)), (n_kv, k, r)
+
+
 def test_split_fed_with_ties(T):
     from oracle import oracle as orc
     rng = np.random.default_rng(1)
