@@ -164,9 +164,13 @@ def test_split_fed_with_ties(T):
         assert right.cpu().tolist() == sorted(order[n_left:])
 
 
-def test_grouping_zero_spread_is_consecutive(T):
-    n, gs = 100, 16
-    Q = torch.ones((1, 2, n, 64), dtype=torch.bfloat16, device="cuda") * 0.375
+@pytest.mark.parametrize("n,d", [(100, 64), (100, 128), (3000, 128)])
+def test_grouping_zero_spread_is_consecutive(T, n, d):
+    # identical rows: every node has zero scatter, its direction is e_0 and
+    # every projection ties, so each cut keeps token order (d = 128 takes the
+    # tensor-core scatter and power iteration, 3000 rows its chunked levels)
+    gs = 16
+    Q = torch.ones((1, 2, n, d), dtype=torch.bfloat16, device="cuda") * 0.375
     ws = T.Workspace(T.dims_of(Q), gs, 1)
     groups = T.group_queries(Q, gs, ws).cpu().numpy()
     G = -(-n // gs)
