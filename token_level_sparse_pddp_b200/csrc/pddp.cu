@@ -421,8 +421,12 @@ __device__ __forceinline__ void split_bf16x2(float d0, float d1, uint32_t& hi, u
 }
 
 // Gram matrix of the rows perm[begin..end) of X ([n_q, 128] bf16, one head)
-// about a shift: TMEM lane a, column b (columns [0,128) at tmem) receives
-// sum_i d_ia d_ib with d_i = x_i - sh.shift. On return sh.m holds the mean of
+// about a shift: sum_i d_ia d_ib with d_i = x_i - sh.shift, split as d = hi +
+// lo (bf16 parts) and taken as hi.hi + hi.lo + lo.hi. TMEM lane a receives
+// hi.hi + lo.hi in columns [0, 128) and hi.lo in columns [128, 256): the first
+// two come from one N = 256 MMA whose B operand is the hi tile followed by the
+// lo tile (an M = 128 MMA costs the same at N = 256 as at N = 128), the third
+// from one N = 128 MMA. On return sh.m holds the mean of
 // d. Thread t handles the 16-byte chunk t % 16 of rows t / 16 + 16 i; the next
 // batch is loaded into registers while the current one is converted and
 // multiplied. Returns false (status recorded, MMAs drained) after a wait that
@@ -472,6 +476,7 @@ __device__ bool gram_tc(const __nv_bfloat16* __restrict__ X, const int32_t* __re
   }
   const uint32_t hi_base = tiles, lo_base = tiles + kTileB;
   constexpr uint32_t idesc = ptx::idesc_bf16(128, 128, true, true);
+  constexpr uint32_t idesc_wide = ptx::idesc_bf16(128, 256, true, true);
   bool ok = true;
   for (int sub = 0; sub < nsub; ++sub) {
     if (sub + 1 < nsub) load(sub + 1, nxt);
@@ -507,10 +512,11 @@ __device__ bool gram_tc(const __nv_bfloat16* __restrict__ X, const int32_t* __re
       ptx::tc_fence_after();
 #pragma unroll
       for (int ks = 0; ks < kSub / 16; ++ks) {
+        // (lo_base = hi_base + 2 * kHalfB: as an N = 256 operand the hi tile's two
+        // 64-channel atoms are followed by the lo tile's)
         const uint64_t dh = ptx::sw128_desc(hi_base + ks * 2048, kHalfB, 1024);
         const uint64_t dl = ptx::sw128_desc(lo_base + ks * 2048, kHalfB, 1024);
-        ptx::mma_ss(tmem, dh, dh, idesc, (sub > 0 || ks > 0) ? 1u : 0u);
-        ptx::mma_ss(tmem, dh, dl, idesc, 1u);
+        ptx::mma_ss(tmem, dh, dh, idesc_wide, (sub > 0 || ks > 0) ? 1u : 0u);
         ptx::mma_ss(tmem, dl, dh, idesc, 1u);
       }
       ptx::tc_commit(&sh.mbar);
@@ -558,7 +564,7 @@ __device__ __forceinline__ uint32_t gram_cta_setup(GramShared& sh) {
     ptx::fence_mbar_init();
   }
   if (threadIdx.x < 32) {
-    ptx::tmem_alloc(&sh.tmem_base, 128);
+    ptx::tmem_alloc(&sh.tmem_base, 256);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
@@ -571,28 +577,30 @@ __device__ __forceinline__ void gram_cta_release(uint32_t tmem) {
   __syncthreads();
   if (threadIdx.x < 32) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, 128);
+    ptx::tmem_dealloc(tmem, 256);
   }
 }
 
 // This thread's 64 entries of the centred scatter held in TMEM: row
-// a = 32 (warp % 4) + lane, columns e0 .. e0 + 63 with e0 = 64 (warp / 4),
-// minus the shift correction n m_a m_b.
+// a = 32 (warp % 4) + lane, columns e0 .. e0 + 63 with e0 = 64 (warp / 4):
+// the sum of the two accumulator halves (hi.hi + lo.hi, and hi.lo), minus the
+// shift correction n m_a m_b.
 __device__ __forceinline__ void gram_row_part(uint32_t tmem, const GramShared& sh, float n,
                                               float (&C)[64]) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int a = 32 * (warp & 3) + lane, e0 = 64 * (warp >> 2);
   const uint32_t tl = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)e0;
-  uint32_t r0[32], r1[32];
-  ptx::tmem_ld32(tl, r0);
-  ptx::tmem_ld32(tl + 32, r1);
-  ptx::tmem_ld_wait(r0);
-  ptx::reg_barrier(r1);
   const float nma = n * sh.m[a];
 #pragma unroll
-  for (int e = 0; e < 32; ++e) {
-    C[e] = __uint_as_float(r0[e]) - nma * sh.m[e0 + e];
-    C[32 + e] = __uint_as_float(r1[e]) - nma * sh.m[e0 + 32 + e];
+  for (int q = 0; q < 4; ++q) {
+    uint32_t l[16], rr[16];
+    ptx::tmem_ld16(tl + 16 * q, l);
+    ptx::tmem_ld16(tl + 128 + 16 * q, rr);
+    ptx::tmem_ld_wait(l);
+    ptx::reg_barrier16(rr);
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+      C[16 * q + e] = (__uint_as_float(l[e]) + __uint_as_float(rr[e])) - nma * sh.m[e0 + 16 * q + e];
   }
 }
 
