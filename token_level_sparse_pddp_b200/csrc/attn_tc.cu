@@ -28,8 +28,9 @@
 // shared-memory slots and V two, so loads run ahead of the math.
 // The softmax keeps a reference max per row and computes each chunk in one
 // pass against it (the first chunk's reference is the max of its first 32
-// columns); only when a chunk's max exceeds the reference by more than 2^8 is
-// the reference raised, O rescaled in TMEM and the chunk recomputed (by the
+// columns); only when the chunk's P sum exceeds 2^8 (no key can exceed the
+// reference by more than 2^8 otherwise) is the chunk's true max taken, the
+// reference raised to it, O rescaled in TMEM and the chunk recomputed (by the
 // whole warp: its TMEM accesses are warp-collective).
 // Between raises the stale reference is used for numerator and denominator
 // alike, which cancels exactly in O / l.

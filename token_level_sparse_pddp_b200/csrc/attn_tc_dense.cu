@@ -19,12 +19,15 @@
 // and O += P_j V_j with A read from TMEM and V as an MN-major B operand.
 // TMEM columns: S double buffer [0,256), O [256,384), P double buffer
 // [384,512), so QK_{j+1} runs while chunk j's softmax does.
-// The softmax keeps a reference max per row and computes each chunk in one
-// pass against it; only when a chunk's max exceeds the reference by more than
-// 2^8 is the reference raised, O rescaled in TMEM and the chunk recomputed
-// (by the whole warp: its TMEM accesses are warp-collective; rows that do not
-// need it keep their reference). Between raises the stale reference is used
-// for numerator and denominator alike, which cancels exactly in O / l.
+// The softmax keeps a reference max per row (the first chunk's: the max of
+// its first 32 columns) and computes each chunk in one pass against it; only
+// when the chunk's P sum exceeds 2^8 (no key can exceed the reference by more
+// than 2^8 otherwise) is the chunk's true max taken, the reference raised to
+// it, O rescaled in TMEM and the chunk recomputed (by the whole warp: its TMEM
+// accesses are warp-collective; rows that do not need it keep their
+// reference, or raise it by less than 2^8). Between raises the stale
+// reference is used for numerator and denominator alike, which cancels
+// exactly in O / l.
 // Every wait is bounded (1 s); on expiry the kernel records
 // TLSP_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 #include <algorithm>
@@ -232,20 +235,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t s_col = tl + kTmS + s * kTile, p_col = tl + kTmP + s * 64;
       // One pass over the chunk in 32-column blocks (the next block's TMEM load
       // in flight while a block is processed): P = 2^(s * scale - m_ref) with
-      // the current reference max, packed to bf16 pairs, while the chunk's
-      // true max is tracked. Returns (sum of P, chunk max).
-      auto p_pass = [&](float m_ref, float& sum_out, float& max_out) {
+      // the current reference max, packed to bf16 pairs. Returns the sum of P.
+      auto p_pass = [&](float m_ref) {
         const float neg_m = -m_ref;
-        float sm[4] = {0.f, 0.f, 0.f, 0.f}, mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        float sm[4] = {0.f, 0.f, 0.f, 0.f};
         auto block = [&](const uint32_t (&cur)[32], int b) {
           uint32_t pk[16];
           if (32 * b + 32 <= valid_n) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const float s0 = __uint_as_float(cur[2 * e]), s1 = __uint_as_float(cur[2 * e + 1]);
-              mx[e & 3] = fmaxf(mx[e & 3], fmaxf(s0, s1));
-              const float p0 = ptx::ex2(fmaf(s0, p.scale_log2, neg_m));
-              const float p1 = ptx::ex2(fmaf(s1, p.scale_log2, neg_m));
+              const float p0 = ptx::ex2(fmaf(__uint_as_float(cur[2 * e]), p.scale_log2, neg_m));
+              const float p1 = ptx::ex2(fmaf(__uint_as_float(cur[2 * e + 1]), p.scale_log2, neg_m));
               sm[e & 3] += p0 + p1;
               pk[e] = pack_bf16(p0, p1);
             }
@@ -253,11 +253,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int c0 = 32 * b + 2 * e;
-              const float s0 = c0 < valid_n ? __uint_as_float(cur[2 * e]) : -INFINITY;
-              const float s1 = c0 + 1 < valid_n ? __uint_as_float(cur[2 * e + 1]) : -INFINITY;
-              mx[e & 3] = fmaxf(mx[e & 3], fmaxf(s0, s1));
-              const float p0 = c0 < valid_n ? ptx::ex2(fmaf(s0, p.scale_log2, neg_m)) : 0.f;
-              const float p1 = c0 + 1 < valid_n ? ptx::ex2(fmaf(s1, p.scale_log2, neg_m)) : 0.f;
+              const float p0 =
+                  c0 < valid_n ? ptx::ex2(fmaf(__uint_as_float(cur[2 * e]), p.scale_log2, neg_m)) : 0.f;
+              const float p1 =
+                  c0 + 1 < valid_n ? ptx::ex2(fmaf(__uint_as_float(cur[2 * e + 1]), p.scale_log2, neg_m))
+                                   : 0.f;
               sm[e & 3] += p0 + p1;
               pk[e] = pack_bf16(p0, p1);
             }
@@ -277,21 +277,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::reg_barrier(rb);
         block(ra, 2);
         block(rb, 3);
-        sum_out = (sm[0] + sm[1]) + (sm[2] + sm[3]);
-        max_out = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        return (sm[0] + sm[1]) + (sm[2] + sm[3]);
       };
-      float sum, mx;
-      bool raise = (j == 0);
-      if (!raise) {
-        p_pass(m_run, sum, mx);  // speculative: usually the reference max still holds
-        // the rescale below is made of warp-collective TMEM accesses, so the
-        // warp takes it together when any of its rows needs it
-        raise = __any_sync(0xffffffffu, mx * p.scale_log2 > m_run + kRescaleLog2);
-      } else {
-        // first chunk: its max becomes the reference
+      // The chunk's max over the valid columns (a pass over S in TMEM, by the
+      // whole warp: `cols` columns).
+      auto max_pass = [&](int cols) {
         float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll 1
-        for (int b = 0; b < 4; ++b) {
+        for (int b = 0; b < cols / 32; ++b) {
           uint32_t c[32];
           ptx::tmem_ld32(s_col + 32 * b, c);
           ptx::tmem_ld_wait(c);
@@ -299,11 +292,22 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 32; ++e)
             if (32 * b + e < valid_n) pm[e & 3] = fmaxf(pm[e & 3], __uint_as_float(c[e]));
         }
-        mx = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
-      }
-      if (raise) {
-        // rows of the warp that do not need it keep their reference (factor 1)
-        const float m_tile = j > 0 ? fmaxf(mx * p.scale_log2, m_run) : mx * p.scale_log2;
+        return fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
+      };
+      // first chunk: the max of its first 32 columns becomes the reference
+      if (j == 0) m_run = max_pass(32) * p.scale_log2;
+      // Speculative: usually the reference still holds. No key of the chunk
+      // exceeds it by more than 2^8 unless the chunk's P sum does, so the sum
+      // decides; only then is the true max taken. The rescale below is made of
+      // warp-collective TMEM accesses, so the warp takes it together when any
+      // of its rows needs it.
+      float sum = p_pass(m_run);
+      // (rows past n_q hold whatever the Q box read there; they never vote, so
+      // a head's result does not depend on the rows that follow it)
+      if (__any_sync(0xffffffffu, tok >= 0 && !(sum <= 256.f))) {
+        // rows of the warp that do not need it keep their reference (factor 1),
+        // or raise it by less than 2^8
+        const float m_tile = fmaxf(max_pass(kTile) * p.scale_log2, m_run);
         if (j > 0) {
           // raise the reference max: O *= 2^(m_run - m_tile) once PV(j-1) has landed
           const float f = ptx::ex2(m_run - m_tile);
@@ -325,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         m_run = m_tile;
         ptx::tmem_st_wait();
-        p_pass(m_run, sum, mx);
+        sum = p_pass(m_run);
       }
       l_run += sum;
       ptx::tmem_st_wait();
