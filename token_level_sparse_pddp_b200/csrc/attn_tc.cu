@@ -481,20 +481,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t s_col = tl + kTmS + s * kTile, p_col = tl + kTmP + s * 64;
       // One pass over the chunk in 32-column blocks (the next block's TMEM load
       // in flight while a block is processed): P = 2^(s * scale - m_ref) with
-      // the current reference max, packed to bf16 pairs. Returns the sum of P.
+      // the current reference max (the scale-and-subtract and the sums on
+      // packed fp32 pairs), packed to bf16 pairs. Returns the sum of P.
       auto p_pass = [&](float m_ref) {
         const float neg_m = -m_ref;
         float sm[4] = {0.f, 0.f, 0.f, 0.f};
+        const uint64_t sc2 = ptx::f2_pack(p.scale_log2, p.scale_log2), nm2 = ptx::f2_pack(neg_m, neg_m);
         auto block = [&](const uint32_t (&cur)[32], int b) {
           uint32_t pk[16];
           if (32 * b + 32 <= valid_n) {
+            uint64_t acc[2] = {0ull, 0ull};
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
-              const float p0 = ptx::ex2(fmaf(__uint_as_float(cur[2 * e]), p.scale_log2, neg_m));
-              const float p1 = ptx::ex2(fmaf(__uint_as_float(cur[2 * e + 1]), p.scale_log2, neg_m));
-              sm[e & 3] += p0 + p1;
+              const uint64_t x = ptx::f2_fma(
+                  ptx::f2_pack(__uint_as_float(cur[2 * e]), __uint_as_float(cur[2 * e + 1])), sc2, nm2);
+              float x0, x1;
+              ptx::f2_unpack(x, x0, x1);
+              const float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
+              acc[e & 1] = ptx::f2_add(acc[e & 1], ptx::f2_pack(p0, p1));
               pk[e] = pack_bf16(p0, p1);
             }
+            float a0, a1, a2, a3;
+            ptx::f2_unpack(acc[0], a0, a1);
+            ptx::f2_unpack(acc[1], a2, a3);
+            sm[b & 3] += (a0 + a1) + (a2 + a3);
           } else {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
