@@ -34,10 +34,12 @@
 // whole warp: its TMEM accesses are warp-collective).
 // Between raises the stale reference is used for numerator and denominator
 // alike, which cancels exactly in O / l.
+// The scale-and-subtract and the row sums run on packed fp32 pairs.
 // Epilogue operands (R rows for the reuse step, O_full rows for the anchor
 // step) are copied by the producers into the two K slots that the last chunk
 // does not use, once those slots' last QK^T has completed, so the epilogue
-// reads them from shared memory instead of waiting on L2 per row.
+// reads them from shared memory instead of waiting on L2 per row; the output
+// rows go back through the free V slots, a whole row per warp store.
 // Every wait is bounded (1 s); on expiry the kernel records
 // TLSP_ERR_TIMEOUT, drains its own copies and MMAs, frees TMEM and returns.
 // Index checks: a selection entry outside [0, n_kv), a group entry outside
