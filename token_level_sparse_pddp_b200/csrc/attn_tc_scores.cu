@@ -14,7 +14,9 @@
 // S^T = K_chunk Q_g^T (M = 128 keys on TMEM lanes, N = 128 queries on TMEM
 // columns), so thread t (lane t) owns key j0 + t and sums its own lane:
 // no cross-thread reduction and no atomics; the per-query LSE (in log2 units)
-// is a shared-memory broadcast. S^T is double-buffered in TMEM so the next
+// is a shared-memory broadcast. A quarter of the exponentials are computed on
+// the FMA pipe (a polynomial, on packed fp32 pairs) instead of the
+// special-function unit, which the pass otherwise saturates. S^T is double-buffered in TMEM so the next
 // chunk's MMA runs while a chunk is summed.
 // Warp roles (416 threads): warps 0-3 sum the even chunks (TMEM buffer 0)
 // and warps 4-7 the odd ones (buffer 1), each lane over all 128 query
@@ -199,10 +201,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     // lane r of warp w is key j * 128 + 32 (w % 4) + r and sums all 128 columns
     const int r = tid & 127, h = warp >> 2;
     if (h == 0) {
-      // log2-unit LSE of the group's queries; padding rows contribute exp2(-inf) = 0
+      // minus the log2-unit LSE of the group's queries; padding rows contribute
+      // exp2(-inf) = 0 (or at most 2.4e-38 on the FMA-pipe path)
       const int tok = r < p.gs ? grp[r] : -1;
-      lse2_s[r] = (tok >= 0 && tok < p.n_q) ? p.lse[bh * p.n_q + tok] * 1.4426950408889634f
-                                             : INFINITY;
+      lse2_s[r] = (tok >= 0 && tok < p.n_q) ? -(p.lse[bh * p.n_q + tok] * 1.4426950408889634f)
+                                             : -INFINITY;
     }
     asm volatile("bar.sync 2, 256;" ::: "memory");
     const float4* l4 = reinterpret_cast<const float4*>(lse2_s);
@@ -214,16 +217,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       ptx::tc_fence_after();
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      uint64_t acc01 = 0ull, acc23 = 0ull;  // packed fp32 pairs
+      const uint64_t sc2 = ptx::f2_pack(p.scale_log2, p.scale_log2);
       // columns 32q .. 32q + 31 of this lane against the queries' LSE
       auto sum32 = [&](const uint32_t (&c)[32], int q) {
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
           const float4 l = l4[(32 * q + e) >> 2];
-          acc[0] += ptx::ex2(fmaf(__uint_as_float(c[e + 0]), p.scale_log2, -l.x));
-          acc[1] += ptx::ex2(fmaf(__uint_as_float(c[e + 1]), p.scale_log2, -l.y));
-          acc[2] += ptx::ex2(fmaf(__uint_as_float(c[e + 2]), p.scale_log2, -l.z));
-          acc[3] += ptx::ex2(fmaf(__uint_as_float(c[e + 3]), p.scale_log2, -l.w));
+          const uint64_t x01 = ptx::f2_fma(ptx::f2_pack(__uint_as_float(c[e]), __uint_as_float(c[e + 1])),
+                                           sc2, ptx::f2_pack(l.x, l.y));
+          const uint64_t x23 = ptx::f2_fma(ptx::f2_pack(__uint_as_float(c[e + 2]), __uint_as_float(c[e + 3])),
+                                           sc2, ptx::f2_pack(l.z, l.w));
+          float a, b;
+          ptx::f2_unpack(x01, a, b);
+          acc01 = ptx::f2_add(acc01, ptx::f2_pack(ptx::ex2(a), ptx::ex2(b)));
+          // every other group of four: its second pair on the FMA pipe, so a
+          // quarter of the exponentials leave the special-function unit
+          if (((e >> 2) % 2) == 2 - 1) {
+            acc23 = ptx::f2_add(acc23, ptx::exp2_poly2(x23));
+          } else {
+            float cc, d;
+            ptx::f2_unpack(x23, cc, d);
+            acc23 = ptx::f2_add(acc23, ptx::f2_pack(ptx::ex2(cc), ptx::ex2(d)));
+          }
         }
       };
       // each quarter's TMEM load is in flight while the one before it is summed
@@ -243,7 +259,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_arrive(&bars.s_empty[h]);  // S is in registers: the MMA may overwrite it
       sum32(c1, 3);
       const int key = j * kTile + r;
-      if (key < p.n_kv) out[key] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      float a0, a1, a2, a3;
+      ptx::f2_unpack(acc01, a0, a1);
+      ptx::f2_unpack(acc23, a2, a3);
+      if (key < p.n_kv) out[key] = (a0 + a1) + (a2 + a3);
     }
   }
 

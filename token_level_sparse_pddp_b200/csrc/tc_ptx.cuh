@@ -313,6 +313,35 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   return d;
 }
 
+// 2^x for a packed pair on the FMA pipe, for x up to 127 (below -125 it reads
+// as -125, whose 2^x is under 2.4e-38): x = n + f with n = round(x) (adding
+// and removing 1.5 * 2^23) and f in [-0.5, 0.5]; 2^f from a degree-5
+// polynomial fitted to 2^f on [-0.5, 0.5] by least squares on Chebyshev
+// nodes with relative weights (max relative error 2.4e-7 in fp32 Horner
+// form); n is then added to the exponent field. It lets part of a kernel's
+// exponentials leave the special-function unit.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t magic = f2_pack(12582912.f, 12582912.f);
+  const uint64_t t = f2_add(x, magic);                                  // 1.5 * 2^23 + round(x)
+  const uint64_t n = f2_add(t, f2_pack(-12582912.f, -12582912.f));      // round(x)
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);                 // x - round(x)
+  uint64_t q = f2_fma(f2_pack(1.3276470e-3f, 1.3276470e-3f), f, f2_pack(9.6755410e-3f, 9.6755410e-3f));
+  q = f2_fma(q, f, f2_pack(5.5507135e-2f, 5.5507135e-2f));
+  q = f2_fma(q, f, f2_pack(2.4022120e-1f, 2.4022120e-1f));
+  q = f2_fma(q, f, f2_pack(6.9314694e-1f, 6.9314694e-1f));
+  q = f2_fma(q, f, f2_pack(1.0000001e+0f, 1.0000001e+0f));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  // the low bits of t hold round(x); shifted into the exponent field they
+  // scale q by 2^round(x) (the 1.5 * 2^23 part shifts out)
+  return f2_pack(__uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23)));
+}
+
 // 2^x on the special-function unit (approximate, relative error ~2^-22).
 __device__ __forceinline__ float ex2(float x) {
   float y;
