@@ -70,7 +70,9 @@ def parse():
 # ----------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi clock / throttle-reason samples during the timed region."""
+    """nvidia-smi clock / throttle-reason samples (every 50 ms) while the GPU is
+    timed: from before the timed steps to after the last timed call (the steps,
+    the separate reuse and dense timings and the end-to-end loop)."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -79,26 +81,48 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.dev = device_index
         self.proc = None
+        self.lines: list[str] = []
+        self.reader = None
 
-    def start(self):
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line)
+
+    def start(self, wait_s: float = 5.0):
+        """Starts the sampler and returns once its first sample has arrived
+        (or after `wait_s`), so the timed region is covered from its start."""
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+            return
+        import atexit
+        atexit.register(self._kill)  # an error between start and stop ends the sampler too
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+        t0 = time.perf_counter()
+        while not self.lines and time.perf_counter() - t0 < wait_s and self.proc.poll() is None:
+            time.sleep(0.01)
+
+    def _kill(self):
+        if self.proc is not None and self.proc.poll() is None:
+            self.proc.kill()
 
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-            out, _ = self.proc.communicate()
-        rows = [r for r in csv.reader(io.StringIO(out)) if len(r) >= 9]
+            self.proc.wait()
+        self.reader.join(timeout=5)
+        rows = [r for r in csv.reader(io.StringIO("".join(self.lines))) if len(r) >= 9]
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
@@ -111,7 +135,8 @@ class ClockSampler:
                 if v.strip().lower() == "active":
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "sm_mhz_min": min(sm) if sm else None}
 
 
 # ----------------------------------------------------------------- CPU oracle leg
@@ -288,7 +313,6 @@ def main():
     torch.cuda.synchronize()
     barrier()
     launches = tlsp.launch_count() - launches0
-    clk = clocks.stop()
     total_ms = t_start.elapsed_time(t_end)
     group_ms = [e[0].elapsed_time(e[1]) for e in events]
     anchor_ms = [e[1].elapsed_time(e[2]) for e in events]
@@ -364,6 +388,7 @@ def main():
             e2e_ev[s - 2][1].record()
     torch.cuda.synchronize()
     e2e_ms = [e[0].elapsed_time(e[1]) for e in e2e_ev]
+    clk = clocks.stop()
     h2d = sum(t.numel() * t.element_size() for t in (Qr_h, Kr_h, Vr_h))
     d2h = O_h.numel() * O_h.element_size()
 

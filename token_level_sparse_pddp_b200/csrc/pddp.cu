@@ -18,6 +18,9 @@
 //   5. split          radix-select cut at rank floor(slots/2)*gs, stable
 //                     partition of the segment (ties: lower token id).
 // After the last level leaf g is the segment [g*gs, (g+1)*gs) of perm.
+// On the tensor-core path, levels whose nodes are handled as one chunk run
+// steps 3-5 in one kernel: a CTA per node builds the scatter, iterates,
+// projects the node's rows and cuts it.
 // bf16 inputs with d = 128 take the tensor-core moments and direction kernels;
 // the other shapes take the fp32 SIMT ones. Both write the same records.
 #include <type_traits>
@@ -405,6 +408,11 @@ struct GramShared {
 constexpr uint32_t kGramSharedB = (sizeof(GramShared) + 1023) / 1024 * 1024;
 constexpr size_t kGramSmem = 1024 + kGramSharedB + 2 * (size_t)kTileB;  // + slack to align
 constexpr size_t kDirSmemNoGram = 1024 + kGramSharedB;
+// A node's level finished inside the direction kernel keeps its order keys at
+// the start of the Gram tiles and the selection state at their end.
+constexpr uint32_t kFuseSelOffset =
+    (2 * kTileB - (uint32_t)sizeof(SelectShared)) / 16 * 16;
+constexpr int kFuseMaxKeys = (int)(kFuseSelOffset / 16 * 4);  // words, a multiple of 4
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -641,17 +649,81 @@ pddp_gram_tc_kernel(const __nv_bfloat16* __restrict__ Q, const int32_t* __restri
   gram_cta_release(tmem);
 }
 
+// Projections of the node's rows perm[off .. off + cnt) on v about the node
+// mean mu = sh.shift + sh.m, with the arithmetic of pddp_project_kernel (16
+// lanes per row, 8 channels each, products summed in channel order, then a
+// shuffle tree), so a projection here is bit-identical to one made there.
+// keys[i] receives the order key of row off + i; trace, when given, the
+// projection at the row's token. Rows just read for the Gram are mostly still
+// in L2; the perm entries of kFuseRows rows are loaded before any of them.
+constexpr int kFuseRows = 8;  // rows per 16-lane group and pass
+__device__ __forceinline__ void project_node_tc(const __nv_bfloat16* __restrict__ X,
+                                                const int32_t* __restrict__ permh, int off,
+                                                int cnt, const GramShared& sh, uint32_t* keys,
+                                                float* __restrict__ trace) {
+  const int sub = threadIdx.x & 15, r0 = threadIdx.x >> 4;
+  float mu[8], vv[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    mu[e] = sh.shift[sub * 8 + e] + sh.m[sub * 8 + e];
+    vv[e] = sh.v[sub * 8 + e];
+  }
+  for (int base = 0; base < cnt; base += (kGT / 16) * kFuseRows) {
+    int tok[kFuseRows];
+#pragma unroll
+    for (int q = 0; q < kFuseRows; ++q) {
+      const int i = base + r0 + (kGT / 16) * q;
+      tok[q] = i < cnt ? permh[off + i] : -1;
+    }
+    float x[kFuseRows][8];
+#pragma unroll
+    for (int q = 0; q < kFuseRows; ++q) {
+      if (tok[q] >= 0) {
+        load8(X + (int64_t)tok[q] * kGD + sub * 8, x[q]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[q][e] = 0.f;
+      }
+    }
+    float pr[kFuseRows];
+#pragma unroll
+    for (int q = 0; q < kFuseRows; ++q) {
+      pr[q] = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) pr[q] = fmaf(x[q][e] - mu[e], vv[e], pr[q]);
+    }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+      for (int q = 0; q < kFuseRows; ++q) pr[q] += __shfl_xor_sync(0xffffffffu, pr[q], o);
+    if (sub == 0) {
+#pragma unroll
+      for (int q = 0; q < kFuseRows; ++q) {
+        if (tok[q] < 0) continue;
+        keys[base + r0 + (kGT / 16) * q] = float_order_key(pr[q]);
+        if (trace) trace[tok[q]] = pr[q];
+      }
+    }
+  }
+}
+
 // Principal direction of one node. With cpn <= 1 the node's scatter is built
 // here (tensor-core Gram over all its rows) and its mean written to node_mu;
 // otherwise both come combined from pddp_reduce_kernel. The scatter stays in
 // registers (thread: row a, 64 columns) for the 16 power iterations
 // v <- C v / |C v|; the sign makes the component of largest magnitude (lowest
 // channel on ties) positive.
+// With `tmp` given (cpn <= 1 only) the kernel also finishes the node's level:
+// the projections of its rows (project_node_tc; trace at trace_level when
+// given), staged as order keys in the Gram tile region, and the cut at rank
+// floor(slots/2)*gs with the stable partition of perm (as pddp_split_smem_kernel,
+// through tmp). The node then needs no projection or split launch.
 __global__ void __launch_bounds__(kGT, 2)
-pddp_direction_tc_kernel(const __nv_bfloat16* __restrict__ Q, const int32_t* __restrict__ perm,
+pddp_direction_tc_kernel(const __nv_bfloat16* __restrict__ Q, int32_t* __restrict__ perm,
                          int n_q, int gs, int G, int level, int cpn, int bh0,
                          const float* __restrict__ partials, float* __restrict__ node_mu,
-                         float* __restrict__ node_v, int* status) {
+                         float* __restrict__ node_v, int* status, int32_t* __restrict__ tmp,
+                         float* __restrict__ trace_level) {
   extern __shared__ uint8_t smem_raw[];
   const GramCta cta = gram_cta_layout(smem_raw);
   GramShared& sh = *cta.sh;
@@ -721,7 +793,29 @@ pddp_direction_tc_kernel(const __nv_bfloat16* __restrict__ Q, const int32_t* __r
     sh.red[4] = sh.v[cmax] < 0.f ? -1.f : 1.f;
   }
   __syncthreads();
-  if (t < kGD) node_v[node * kGD + t] = sh.v[t] * sh.red[4];
+  const float vf = t < kGD ? sh.v[t] * sh.red[4] : 0.f;
+  if (t < kGD) node_v[node * kGD + t] = vf;
+  if (tmp == nullptr || cpn > 1) return;
+  __syncthreads();  // every thread has read sh.v and sh.red[4]
+  if (t < kGD) sh.v[t] = vf;
+  // keys, then the selection state, in the Gram tiles (their MMAs completed)
+  uint8_t* tiles = smem_raw + (cta.tiles - ptx::smem_u32(smem_raw));
+  uint32_t* keys = reinterpret_cast<uint32_t*>(tiles);
+  SelectShared& ssh = *reinterpret_cast<SelectShared*>(tiles + kFuseSelOffset);
+  __syncthreads();
+  const int64_t base = (int64_t)bh * n_q + nd.off;
+  project_node_tc(Q + (int64_t)bh * n_q * kGD, perm + (int64_t)bh * n_q, nd.off, nd.cnt, sh, keys,
+                  trace_level ? trace_level + (int64_t)bh * n_q : nullptr);
+  __syncthreads();
+  const int n_left = (nd.slots / 2) * gs;
+  int32_t* p = perm + base;
+  int32_t* o = tmp + base;
+  smem_select_ordered<kGT>(
+      keys, nd.cnt, n_left, [](uint32_t w) { return w; }, ssh,
+      [&](uint32_t pos, int i) { o[pos] = p[i]; },
+      [&](uint32_t pos, int i) { o[n_left + pos] = p[i]; });
+  __syncthreads();
+  for (int i = t; i < nd.cnt; i += kGT) p[i] = o[i];
 }
 
 // pddp_split_kernel with the node's keys staged in shared memory (nodes of
@@ -806,6 +900,8 @@ static int run_pddp_t(const T* Q, int64_t BH, int n_q, int gs, int32_t* groups, 
     int64_t cpn = kTc ? ceil_div(max_rows, 2 * kSub) : ceil_div(max_rows, 256);
     cpn = std::min<int64_t>(cpn, std::max<int64_t>(1, kChunksPerHead / nodes));
     if (cpn < 2) cpn = 1;
+    // levels whose nodes build their own scatter also project and cut them there
+    const bool fused = kTc && cpn == 1 && max_rows <= kFuseMaxKeys;
     // heads whose chunk records fit in the workspace at once
     const int64_t hb = cpn > 1 ? std::max<int64_t>(1, w.partial_slots / (nodes * cpn)) : BH;
     for (int64_t h0 = 0; h0 < BH; h0 += hb) {
@@ -829,7 +925,7 @@ static int run_pddp_t(const T* Q, int64_t BH, int n_q, int gs, int32_t* groups, 
         pddp_direction_tc_kernel<<<dim3((unsigned)nodes, nh), kGT,
                                    cpn > 1 ? kDirSmemNoGram : kGramSmem, st>>>(
             Q, w.perm, n_q, gs, G, level, (int)cpn, (int)h0, w.partials, w.node_mu, w.node_v,
-            w.status);
+            w.status, fused ? w.tmp : nullptr, fused && trace ? trace + level * total : nullptr);
       } else {
         pddp_direction_kernel<T, D><<<dim3((unsigned)nodes, nh), kMomThreads,
                                       direction_smem_bytes<D>(), st>>>(
@@ -837,6 +933,7 @@ static int run_pddp_t(const T* Q, int64_t BH, int n_q, int gs, int32_t* groups, 
       }
       TLSP_TRY(check_launch());
     }
+    if (fused) continue;
     constexpr int kRowsPerBlock = 256 / (D * (int)sizeof(T) / 16) * kProjRows;
     pddp_project_kernel<T, D>
         <<<dim3((unsigned)ceil_div(n_q, kRowsPerBlock), (unsigned)BH), 256, 0, st>>>(

@@ -24,11 +24,14 @@ struct SelectShared {
 };
 
 // Locates the bin of sh.hist where the running count reaches `rank`
-// (1-based): sh.bcast[0] = bin, sh.bcast[1] = rank within that bin. Each
-// thread owns kRadixBins / kSelectThreads consecutive bins; a block scan of the
-// per-thread sums finds the owner. Ends with a barrier.
+// (1-based): sh.bcast[0] = bin, sh.bcast[1] = rank within that bin. Each of
+// the block's NT threads (at most kSelectThreads) owns kRadixBins / NT
+// consecutive bins; a block scan of the per-thread sums finds the owner. Ends
+// with a barrier.
+template <int NT = kSelectThreads>
 __device__ __forceinline__ void find_rank_bin(SelectShared& sh, uint32_t rank) {
-  constexpr int per = kRadixBins / kSelectThreads;
+  static_assert(NT % 32 == 0 && NT <= kSelectThreads && kRadixBins % NT == 0, "block size");
+  constexpr int per = kRadixBins / NT;
   uint32_t local[per], lsum = 0;
 #pragma unroll
   for (int q = 0; q < per; ++q) {
@@ -165,15 +168,15 @@ __device__ void select_smallest_ordered(KeyFn key, int n, int m, SelectShared& s
 // passes over contiguous per-warp ranges: per-lane counts, then, per 128
 // positions, four ballots whose popcounts give every member its offset.
 
-template <class KeyOf>
+template <int NT, class KeyOf>
 __device__ void smem_radix_select(uint32_t* w, int n, int m, KeyOf key_of, SelectShared& sh,
                                   uint32_t* T, int* need_eq) {
   const int t = threadIdx.x;
   const int n4 = n >> 2;
   uint4* w4 = reinterpret_cast<uint4*>(w);
-  for (int b = t; b < kRadixBins; b += kSelectThreads) sh.hist[b] = 0;
+  for (int b = t; b < kRadixBins; b += NT) sh.hist[b] = 0;
   __syncthreads();
-  for (int v = t; v < n4; v += kSelectThreads) {
+  for (int v = t; v < n4; v += NT) {
     uint4 u = w4[v];
     u.x = key_of(u.x);
     u.y = key_of(u.y);
@@ -185,12 +188,12 @@ __device__ void smem_radix_select(uint32_t* w, int n, int m, KeyOf key_of, Selec
     atomicAdd(&sh.hist[u.z >> 21], 1u);
     atomicAdd(&sh.hist[u.w >> 21], 1u);
   }
-  for (int i = 4 * n4 + t; i < n; i += kSelectThreads) {
+  for (int i = 4 * n4 + t; i < n; i += NT) {
     w[i] = key_of(w[i]);
     atomicAdd(&sh.hist[w[i] >> 21], 1u);
   }
   __syncthreads();
-  find_rank_bin(sh, (uint32_t)m);
+  find_rank_bin<NT>(sh, (uint32_t)m);
   uint32_t prefix = sh.bcast[0];  // top 11 bits
   uint32_t rank = sh.bcast[1];
   __syncthreads();
@@ -198,19 +201,19 @@ __device__ void smem_radix_select(uint32_t* w, int n, int m, KeyOf key_of, Selec
     const int shift = pass == 1 ? 21 : 10;  // keys match when k >> shift == prefix
     const int dshift = pass == 1 ? 10 : 0;
     const uint32_t dmask = pass == 1 ? 0x7ffu : 0x3ffu;
-    for (int b = t; b < kRadixBins; b += kSelectThreads) sh.hist[b] = 0;
+    for (int b = t; b < kRadixBins; b += NT) sh.hist[b] = 0;
     __syncthreads();
-    for (int v = t; v < n4; v += kSelectThreads) {
+    for (int v = t; v < n4; v += NT) {
       const uint4 u = w4[v];
       if ((u.x >> shift) == prefix) atomicAdd(&sh.hist[(u.x >> dshift) & dmask], 1u);
       if ((u.y >> shift) == prefix) atomicAdd(&sh.hist[(u.y >> dshift) & dmask], 1u);
       if ((u.z >> shift) == prefix) atomicAdd(&sh.hist[(u.z >> dshift) & dmask], 1u);
       if ((u.w >> shift) == prefix) atomicAdd(&sh.hist[(u.w >> dshift) & dmask], 1u);
     }
-    for (int i = 4 * n4 + t; i < n; i += kSelectThreads)
+    for (int i = 4 * n4 + t; i < n; i += NT)
       if ((w[i] >> shift) == prefix) atomicAdd(&sh.hist[(w[i] >> dshift) & dmask], 1u);
     __syncthreads();
-    find_rank_bin(sh, rank);
+    find_rank_bin<NT>(sh, rank);
     prefix = (prefix << (pass == 1 ? 11 : 10)) | sh.bcast[0];
     rank = sh.bcast[1];
     __syncthreads();
@@ -221,16 +224,18 @@ __device__ void smem_radix_select(uint32_t* w, int n, int m, KeyOf key_of, Selec
 
 // Selects the m smallest keys among the n staged words (ties to the lower
 // position), emitting sel(pos_in_selection, i) and rest(pos_in_rest, i) in
-// position order. 0 <= m <= n. The words are replaced by their keys.
-template <class KeyOf, class SelFn, class RestFn>
+// position order. 0 <= m <= n. The words are replaced by their keys. NT is the
+// block's thread count (a multiple of 32, at most kSelectThreads); the result
+// does not depend on it.
+template <int NT = kSelectThreads, class KeyOf, class SelFn, class RestFn>
 __device__ void smem_select_ordered(uint32_t* w, int n, int m, KeyOf key_of, SelectShared& sh,
                                     SelFn sel, RestFn rest) {
-  constexpr int W = kSelectThreads / 32;
+  constexpr int W = NT / 32;
   const bool take_all = (m >= n), take_none = (m <= 0);
   const bool cut = !take_all && !take_none;
   uint32_t T = 0;
   int need_eq = 0;
-  if (cut) smem_radix_select(w, n, m, key_of, sh, &T, &need_eq);
+  if (cut) smem_radix_select<NT>(w, n, m, key_of, sh, &T, &need_eq);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t below = (1u << lane) - 1u;
   const int n_slots = (n + 3) >> 2;
