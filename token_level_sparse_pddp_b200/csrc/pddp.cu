@@ -355,6 +355,33 @@ pddp_project_kernel(const T* __restrict__ Q, const int32_t* __restrict__ perm, i
   }
 }
 
+// Applies a cut to a node's perm segment p[0 .. n): o[j] is the index in p of
+// the token that goes to position j (the ordered selection writes indices, not
+// tokens, so it issues no load). The tokens are gathered into the staging
+// words w (shared memory, n words, free by now) kGatherUnroll at a time, all
+// loads before any store, and then written back; no global load waits on a
+// global store. NT is the block's thread count.
+constexpr int kGatherUnroll = 8;
+template <int NT>
+__device__ __forceinline__ void apply_partition(int32_t* p, const int32_t* o, uint32_t* w, int n) {
+  for (int j0 = threadIdx.x; j0 < n; j0 += kGatherUnroll * NT) {
+    int src[kGatherUnroll];
+#pragma unroll
+    for (int u = 0; u < kGatherUnroll; ++u) {
+      const int j = j0 + u * NT;
+      src[u] = j < n ? min(max(o[j], 0), n - 1) : 0;  // (in range by construction)
+    }
+    int32_t val[kGatherUnroll];
+#pragma unroll
+    for (int u = 0; u < kGatherUnroll; ++u) val[u] = p[src[u]];
+#pragma unroll
+    for (int u = 0; u < kGatherUnroll; ++u)
+      if (j0 + u * NT < n) w[j0 + u * NT] = (uint32_t)val[u];
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < n; j += NT) p[j] = (int32_t)w[j];
+}
+
 // One CTA per split node: cut at rank floor(slots/2)*gs on the segment keys,
 // stable partition into tmp, then copy back into perm.
 __global__ void __launch_bounds__(kSelectThreads)
@@ -786,11 +813,25 @@ pddp_direction_tc_kernel(const __nv_bfloat16* __restrict__ Q, int32_t* __restric
     if (t < kGD) sh.v[t] = w / nw;
     __syncthreads();
   }
-  if (t == 0) {
-    int cmax = 0;
-    for (int c = 1; c < kGD; ++c)
-      if (fabsf(sh.v[c]) > fabsf(sh.v[cmax])) cmax = c;
-    sh.red[4] = sh.v[cmax] < 0.f ? -1.f : 1.f;
+  if (warp == 0) {  // component of largest magnitude, lowest channel on ties
+    float best = fabsf(sh.v[lane]);
+    int cmax = lane;
+#pragma unroll
+    for (int c = lane + 32; c < kGD; c += 32)
+      if (fabsf(sh.v[c]) > best) {
+        best = fabsf(sh.v[c]);
+        cmax = c;
+      }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oc = __shfl_xor_sync(0xffffffffu, cmax, o);
+      if (ob > best || (ob == best && oc < cmax)) {
+        best = ob;
+        cmax = oc;
+      }
+    }
+    if (lane == 0) sh.red[4] = sh.v[cmax] < 0.f ? -1.f : 1.f;
   }
   __syncthreads();
   const float vf = t < kGD ? sh.v[t] * sh.red[4] : 0.f;
@@ -812,15 +853,16 @@ pddp_direction_tc_kernel(const __nv_bfloat16* __restrict__ Q, int32_t* __restric
   int32_t* o = tmp + base;
   smem_select_ordered<kGT>(
       keys, nd.cnt, n_left, [](uint32_t w) { return w; }, ssh,
-      [&](uint32_t pos, int i) { o[pos] = p[i]; },
-      [&](uint32_t pos, int i) { o[n_left + pos] = p[i]; });
+      [&](uint32_t pos, int i) { o[pos] = i; },
+      [&](uint32_t pos, int i) { o[n_left + pos] = i; });
   __syncthreads();
-  for (int i = t; i < nd.cnt; i += kGT) p[i] = o[i];
+  apply_partition<kGT>(p, o, keys, nd.cnt);
 }
 
 // pddp_split_kernel with the node's keys staged in shared memory (nodes of
-// at most kSplitSmemKeys tokens). Dynamic shared memory: keys rounded up to 4
-// words.
+// at most kSplitSmemKeys tokens); the selection writes indices into tmp and
+// apply_partition moves the tokens. Dynamic shared memory: keys rounded up to
+// 4 words.
 constexpr int kSplitSmemKeys = 52 * 1024;
 __global__ void __launch_bounds__(kSelectThreads)
 pddp_split_smem_kernel(int32_t* __restrict__ perm, int32_t* __restrict__ tmp,
@@ -839,10 +881,10 @@ pddp_split_smem_kernel(int32_t* __restrict__ perm, int32_t* __restrict__ tmp,
   int32_t* o = tmp + base;
   smem_select_ordered(
       keys, nd.cnt, n_left, [](uint32_t w) { return w; }, sh,
-      [&](uint32_t pos, int i) { o[pos] = p[i]; },
-      [&](uint32_t pos, int i) { o[n_left + pos] = p[i]; });
+      [&](uint32_t pos, int i) { o[pos] = i; },
+      [&](uint32_t pos, int i) { o[n_left + pos] = i; });
   __syncthreads();
-  for (int i = threadIdx.x; i < nd.cnt; i += kSelectThreads) p[i] = o[i];
+  apply_partition<kSelectThreads>(p, o, keys, nd.cnt);
 }
 
 __global__ void pddp_init_kernel(int32_t* __restrict__ perm, int n_q, int64_t total) {
