@@ -734,6 +734,119 @@ __device__ __forceinline__ void project_node_tc(const __nv_bfloat16* __restrict_
   }
 }
 
+// Node of position pos at `level` (as pddp_project_kernel walks it); false
+// for positions in leaves made at earlier levels.
+__device__ __forceinline__ bool live_node_of(int pos, int n_q, int gs, int G, int level, int& j) {
+  int off = 0, slots = G;
+  j = 0;
+  if (pos >= n_q) return false;
+  for (int b = 0; b < level; ++b) {
+    if (slots == 1) return false;
+    const int ls = slots / 2, boundary = off + ls * gs;
+    if (pos < boundary) {
+      slots = ls;
+      j = 2 * j;
+    } else {
+      off = boundary;
+      slots -= ls;
+      j = 2 * j + 1;
+    }
+  }
+  return slots > 1;
+}
+
+// pddp_project_kernel for bf16 rows of 128 channels, restructured for memory
+// parallelism: each 16-lane group walks runs of kProjRun consecutive positions
+// of one head (grid-stride), loading the next run's perm entries while the
+// current run's rows are in flight, and keeps its node's mean and direction in
+// registers while the positions stay in that node. A warp takes two runs per
+// step (one per half) and steps while its first run is in range, so every
+// shuffle has all 32 lanes. Per row the arithmetic is that of
+// pddp_project_kernel, so the keys are bit-identical. Grid: (blocks per head,
+// BH).
+constexpr int kProjRun = 8;
+constexpr int kProjBlocksPerSm = 3;
+__global__ void __launch_bounds__(256, kProjBlocksPerSm)
+pddp_project_tc_kernel(const __nv_bfloat16* __restrict__ Q, const int32_t* __restrict__ perm,
+                       int n_q, int gs, int G, int level, const float* __restrict__ node_mu,
+                       const float* __restrict__ node_v, uint32_t* __restrict__ seg_key,
+                       float* __restrict__ trace, int64_t trace_level_stride) {
+  const int sub = threadIdx.x & 15, half = (threadIdx.x >> 4) & 1, bh = blockIdx.y;
+  const int wg = blockIdx.x * 8 + (threadIdx.x >> 5), step = gridDim.x * 16;
+  const int nrun = (n_q + kProjRun - 1) / kProjRun;
+  const int32_t* ph = perm + (int64_t)bh * n_q;
+  const uint4* Xh = reinterpret_cast<const uint4*>(Q + (int64_t)bh * n_q * kGD);
+  const float* mu_h = node_mu + (int64_t)bh * G * kGD + sub * 8;
+  const float* v_h = node_v + (int64_t)bh * G * kGD + sub * 8;
+  int tok[kProjRun];
+  auto fetch = [&](int run) {
+#pragma unroll
+    for (int q = 0; q < kProjRun; ++q) {
+      const int pos = run * kProjRun + q;
+      tok[q] = (run < nrun && pos < n_q) ? ph[pos] : -1;
+    }
+  };
+  fetch(2 * wg + half);
+  int cur = -1;
+  float mu[8], vv[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) mu[e] = vv[e] = 0.f;
+  for (int base = 2 * wg; base < nrun; base += step) {  // (warp-uniform)
+    const int run = base + half;
+    uint4 raw[kProjRun];
+    int tk[kProjRun];
+#pragma unroll
+    for (int q = 0; q < kProjRun; ++q) {
+      tk[q] = tok[q];
+      raw[q] = tk[q] >= 0 ? __ldg(Xh + (int64_t)tk[q] * (kGD / 8) + sub) : make_uint4(0, 0, 0, 0);
+    }
+    fetch(run + step);  // in flight with the rows above
+    const int p0 = run * kProjRun;
+    int j_first, j_last;
+    const bool l_first = live_node_of(p0, n_q, gs, G, level, j_first);
+    const bool l_last = live_node_of(min(p0 + kProjRun, n_q) - 1, n_q, gs, G, level, j_last);
+    const bool one_node = l_first && l_last && j_first == j_last;
+    float pr[kProjRun];
+    bool live[kProjRun];
+#pragma unroll
+    for (int q = 0; q < kProjRun; ++q) {
+      int j = j_first;
+      live[q] = tk[q] >= 0 && (one_node || live_node_of(p0 + q, n_q, gs, G, level, j));
+      pr[q] = 0.f;
+      if (!live[q]) continue;
+      if (j != cur) {
+        const float4 m0 = *reinterpret_cast<const float4*>(mu_h + (int64_t)j * kGD);
+        const float4 m1 = *reinterpret_cast<const float4*>(mu_h + (int64_t)j * kGD + 4);
+        const float4 v0 = *reinterpret_cast<const float4*>(v_h + (int64_t)j * kGD);
+        const float4 v1 = *reinterpret_cast<const float4*>(v_h + (int64_t)j * kGD + 4);
+        mu[0] = m0.x; mu[1] = m0.y; mu[2] = m0.z; mu[3] = m0.w;
+        mu[4] = m1.x; mu[5] = m1.y; mu[6] = m1.z; mu[7] = m1.w;
+        vv[0] = v0.x; vv[1] = v0.y; vv[2] = v0.z; vv[3] = v0.w;
+        vv[4] = v1.x; vv[5] = v1.y; vv[6] = v1.z; vv[7] = v1.w;
+        cur = j;
+      }
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t w = word_of(raw[q], k);
+        pr[q] = fmaf(bf16_lo(w) - mu[2 * k], vv[2 * k], pr[q]);
+        pr[q] = fmaf(bf16_hi(w) - mu[2 * k + 1], vv[2 * k + 1], pr[q]);
+      }
+    }
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1)
+#pragma unroll
+      for (int q = 0; q < kProjRun; ++q) pr[q] += __shfl_xor_sync(0xffffffffu, pr[q], o);
+    if (sub == 0) {
+#pragma unroll
+      for (int q = 0; q < kProjRun; ++q) {
+        if (!live[q]) continue;
+        seg_key[(int64_t)bh * n_q + p0 + q] = float_order_key(pr[q]);
+        if (trace) trace[level * trace_level_stride + (int64_t)bh * n_q + tk[q]] = pr[q];
+      }
+    }
+  }
+}
+
 // Principal direction of one node. With cpn <= 1 the node's scatter is built
 // here (tensor-core Gram over all its rows) and its mean written to node_mu;
 // otherwise both come combined from pddp_reduce_kernel. The scatter stays in
@@ -976,10 +1089,20 @@ static int run_pddp_t(const T* Q, int64_t BH, int n_q, int gs, int32_t* groups, 
       TLSP_TRY(check_launch());
     }
     if (fused) continue;
-    constexpr int kRowsPerBlock = 256 / (D * (int)sizeof(T) / 16) * kProjRows;
-    pddp_project_kernel<T, D>
-        <<<dim3((unsigned)ceil_div(n_q, kRowsPerBlock), (unsigned)BH), 256, 0, st>>>(
-            Q, w.perm, n_q, gs, G, level, w.node_mu, w.node_v, w.seg_key, trace, total);
+    if constexpr (kTc) {
+      // one resident wave of blocks in all, at most one 16-lane group per run
+      const int64_t runs = ceil_div(n_q, kProjRun);
+      const int64_t per_head = std::max<int64_t>(
+          1, std::min<int64_t>(ceil_div(kProjBlocksPerSm * (int64_t)device_sm_count(), BH),
+                               ceil_div(runs, 16)));
+      pddp_project_tc_kernel<<<dim3((unsigned)per_head, (unsigned)BH), 256, 0, st>>>(
+          Q, w.perm, n_q, gs, G, level, w.node_mu, w.node_v, w.seg_key, trace, total);
+    } else {
+      constexpr int kRowsPerBlock = 256 / (D * (int)sizeof(T) / 16) * kProjRows;
+      pddp_project_kernel<T, D>
+          <<<dim3((unsigned)ceil_div(n_q, kRowsPerBlock), (unsigned)BH), 256, 0, st>>>(
+              Q, w.perm, n_q, gs, G, level, w.node_mu, w.node_v, w.seg_key, trace, total);
+    }
     TLSP_TRY(check_launch());
     if (max_rows <= kSplitSmemKeys) {
       const size_t smem = (size_t)((max_rows + 3) & ~3) * 4;
