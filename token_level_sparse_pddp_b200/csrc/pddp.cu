@@ -464,8 +464,9 @@ __device__ __forceinline__ void split_bf16x2(float d0, float d1, uint32_t& hi, u
 // from one N = 128 MMA. On return sh.m holds the mean of
 // d. Thread t handles the 16-byte chunk t % 16 of rows t / 16 + 16 i; the next
 // batch is loaded into registers while the current one is converted and
-// multiplied. Returns false (status recorded, MMAs drained) after a wait that
-// ran out; the result is the same for every thread of the block.
+// multiplied, and the perm entries of the batch after it are loaded with it.
+// Returns false (status recorded, MMAs drained) after a wait that ran out; the
+// result is the same for every thread of the block.
 __device__ bool gram_tc(const __nv_bfloat16* __restrict__ X, const int32_t* __restrict__ perm,
                         int begin, int end, uint32_t tiles, GramShared& sh, uint32_t tmem,
                         int* status) {
@@ -476,14 +477,22 @@ __device__ bool gram_tc(const __nv_bfloat16* __restrict__ X, const int32_t* __re
   const int nsub = (n + kSub - 1) / kSub;
   const uint4* Xv = reinterpret_cast<const uint4*>(X);
   uint4 cur[8], nxt[8];
-  auto load = [&](int sub, uint4(&buf)[8]) {
+  int ix[8];  // perm entries of the next batch whose rows are not yet requested
+  auto fetch = [&](int sub) {
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int r = begin + sub * kSub + ro + 16 * i;
-      buf[i] = r < end ? __ldg(Xv + (int64_t)perm[r] * (kGD / 8) + q) : make_uint4(0, 0, 0, 0);
+      ix[i] = (sub < nsub && r < end) ? perm[r] : -1;
     }
   };
-  load(0, cur);
+  auto load = [&](uint4(&buf)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      buf[i] = ix[i] >= 0 ? __ldg(Xv + (int64_t)ix[i] * (kGD / 8) + q) : make_uint4(0, 0, 0, 0);
+  };
+  fetch(0);
+  load(cur);
+  fetch(1);
   {  // shift: mean of the first batch (rows past the end load as zeros)
     float s[8] = {};
 #pragma unroll
@@ -514,7 +523,10 @@ __device__ bool gram_tc(const __nv_bfloat16* __restrict__ X, const int32_t* __re
   constexpr uint32_t idesc_wide = ptx::idesc_bf16(128, 256, true, true);
   bool ok = true;
   for (int sub = 0; sub < nsub; ++sub) {
-    if (sub + 1 < nsub) load(sub + 1, nxt);
+    if (sub + 1 < nsub) {
+      load(nxt);       // rows of batch sub + 1 (their perm entries arrived a batch ago)
+      fetch(sub + 2);  // perm entries of batch sub + 2, in flight with those rows
+    }
     // the tile is rewritten only after the previous batch's MMAs have read it
     if (sub > 0) ok = ptx::mbar_wait(&sh.mbar, (sub - 1) & 1, nullptr, kGramWaitNs);
     if (ok) {
